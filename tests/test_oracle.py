@@ -1,0 +1,432 @@
+"""Pins for the CPU oracle against things other than itself.
+
+Each test names what fixes the expected value: a number printed on the pages
+(tests/golden/worked_example.txt), a closed form, exact rational brute force,
+an independent library routine (scipy's normal CDF, torch's bf16 cast,
+torch.autograd), or an invariant the method must satisfy.  CPU only.
+"""
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import ndtr
+
+import oracle
+from oracle import nf4 as O
+
+
+# ---------------------------------------------------------------------------
+# NF4 table
+# ---------------------------------------------------------------------------
+
+def test_nf4_table_structure():
+    """'That is NF4': 16 values, one exactly 0, spanning [-1, 1]."""
+    q = oracle.nf4_table()
+    assert q.dtype == np.float32 and q.shape == (16,)
+    assert np.all(np.diff(q) > 0)
+    assert q[0] == -1.0 and q[15] == 1.0
+    assert q[7] == 0.0 and np.count_nonzero(q == 0) == 1
+    assert np.sum(q < 0) == 7 and np.sum(q > 0) == 8
+
+
+def test_nf4_table_is_normal_quantiles():
+    """The positive levels sit at evenly spaced probabilities of N(0,1), from
+    1/2 up to 1 - delta; the negative ones likewise with one level fewer.
+    Checked with scipy's forward CDF (ndtr), not the inverse used to build it."""
+    q = oracle.nf4_table().astype(np.float64)
+    delta = 0.5 * (1 / 30 + 1 / 32)
+    zmax = None
+    # un-normalise with the top quantile: Phi(zmax) = 1 - delta
+    lo, hi = 0.0, 10.0
+    for _ in range(200):
+        mid = (lo + hi) / 2
+        lo, hi = (mid, hi) if ndtr(mid) < 1 - delta else (lo, mid)
+    zmax = lo
+    pos = ndtr(q[8:] * zmax)                 # 8 positive levels, ascending
+    neg = ndtr(-q[:7] * zmax)                # 7 negative levels, descending mass
+    # fp32 rounding of q moves Phi by at most ~ pdf * zmax * 2^-24 * |q|
+    assert np.allclose(np.diff(np.concatenate([[0.5], pos])), (1 - delta - 0.5) / 8, atol=2e-7)
+    assert np.allclose(np.diff(np.concatenate([[0.5], neg[::-1]])), (1 - delta - 0.5) / 7, atol=2e-7)
+
+
+def test_nf4_finer_near_zero():
+    """'The steps are noticeably finer near zero ... coarser out in the tails'."""
+    q = oracle.nf4_table().astype(np.float64)
+    gaps_pos = np.diff(q[7:])
+    gaps_neg = np.diff(q[:8])[::-1]
+    assert np.all(np.diff(gaps_pos) > 0)
+    assert np.all(np.diff(gaps_neg) > 0)
+    assert gaps_pos[0] < 2 / 15 and gaps_neg[0] < 2 / 15
+
+
+def test_nf4_beats_uniform_on_gaussian_weights():
+    """'Same four bits ... buys back a large part of the accuracy that even
+    spacing threw away' (That is NF4); NF4 beats uniform INT4 (quiz page)."""
+    rng = np.random.default_rng(7)
+    W = (rng.standard_normal((256, 1024)) * 0.02).astype(np.float32)
+    errs = {}
+    for name, table in (("nf4", oracle.nf4_table()), ("uniform", oracle.uniform_table())):
+        codes, a = oracle.quantize(W, table)
+        Wd = oracle.dequantize(oracle.pack(codes), a, W.shape, table)
+        errs[name] = float(np.sqrt(np.mean((Wd - W) ** 2)))
+    assert errs["nf4"] < 0.95 * errs["uniform"]
+
+
+# ---------------------------------------------------------------------------
+# Nearest code: thresholds vs exact rational brute force
+# ---------------------------------------------------------------------------
+
+def _brute_code(x: float, table) -> int:
+    """argmin_i |x - q_i| in exact rationals; ties -> higher index."""
+    fx = Fraction(float(x))
+    best, bi = None, -1
+    for i, qi in enumerate(table):
+        d = abs(fx - Fraction(float(qi)))
+        if best is None or d <= best:
+            best, bi = d, i
+    return bi
+
+
+@pytest.mark.parametrize("table_name", ["nf4", "uniform"])
+def test_threshold_code_equals_brute_force(table_name):
+    table = oracle.nf4_table() if table_name == "nf4" else oracle.uniform_table()
+    xs = []
+    q = table.astype(np.float64)
+    for j in range(15):
+        m = np.float32((q[j] + q[j + 1]) / 2)
+        v = m
+        for _ in range(5):
+            v = np.nextafter(v, np.float32(-2))
+        for _ in range(11):
+            xs.append(v)
+            v = np.nextafter(v, np.float32(2))
+    rng = np.random.default_rng(3)
+    xs += list(rng.uniform(-1, 1, 2000).astype(np.float32))
+    xs += [np.float32(v) for v in (-1.0, 1.0, 0.0, -0.0)] + list(table)
+    xs = np.array(xs, dtype=np.float32)
+    got = oracle.nearest_code(xs, table)
+    want = np.array([_brute_code(x, table) for x in xs])
+    assert np.array_equal(got, want)
+
+
+def test_quantize_tiny_blocks_brute_force():
+    """Whole quantise path on tiny random blocks vs rational brute force."""
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((4, 128)) * 0.02).astype(np.float32)
+    table = oracle.nf4_table()
+    codes, a = oracle.quantize(W, table)
+    blk = W.reshape(-1, 64)
+    assert np.array_equal(a, np.abs(blk).max(axis=1))
+    for b in range(blk.shape[0]):
+        for i in range(64):
+            x = np.float32(blk[b, i]) / np.float32(a[b])       # RN32 division
+            assert codes[64 * b + i] == _brute_code(x, table)
+
+
+# ---------------------------------------------------------------------------
+# The pages' worked example, uniform table
+# ---------------------------------------------------------------------------
+
+def _example_block(values, scale=0.08):
+    blk = np.zeros(64, dtype=np.float32)
+    blk[0] = np.float32(scale)
+    blk[1:1 + len(values)] = np.array(values, dtype=np.float32)
+    return blk.reshape(1, 64)
+
+
+def test_worked_example_uniform_table(golden):
+    g = golden
+    u = oracle.uniform_table()
+    assert u[1] - u[0] == pytest.approx(g["uniform_step"], abs=5e-4)
+    assert u[1] == pytest.approx(g["uniform_row_1"], abs=5e-4)
+    assert u[2] == pytest.approx(g["uniform_row_2"], abs=5e-4)
+
+    W = _example_block([g["example_w"], g["small_w"], 0.0])
+    codes, a = oracle.quantize(W, u)
+    assert a[0] == np.float32(g["example_scale"])
+    x = oracle.normalise(W, a)[0]
+    assert x[1] == pytest.approx(g["example_x"], abs=5e-4)
+    assert x[2] == pytest.approx(g["small_x"], abs=5e-5)
+    # step 3: nearest rows
+    assert u[codes[1]] == pytest.approx(g["example_row"], abs=5e-4)
+    assert u[codes[1] - 1] == pytest.approx(g["example_lower_row"], abs=5e-4)
+    assert (u[codes[2] - 1], u[codes[2]]) == pytest.approx(g["small_rows"], abs=5e-5)
+    # step 4 and the two failures: read back = row * scale (fp32, before bf16)
+    back = (u[codes] * a[0]).astype(np.float32)
+    assert back[1] == pytest.approx(g["example_back"], abs=5e-5)
+    assert abs(back[1] - g["example_w"]) == pytest.approx(g["example_loss"], abs=5e-5)
+    assert back[2] == pytest.approx(g["small_back"], abs=5e-5)
+    assert abs(back[2] - g["small_w"]) / g["small_w"] == pytest.approx(g["small_rel_err"], abs=5e-3)
+    # zero lands exactly between the two middle rows and goes up
+    assert codes[3] == 8
+    assert back[3] == pytest.approx(g["zero_back"], abs=5e-5)
+
+
+# ---------------------------------------------------------------------------
+# Quantise invariants
+# ---------------------------------------------------------------------------
+
+def test_zero_block_and_signed_zero():
+    W = np.zeros((1, 128), dtype=np.float32)
+    W[0, 64] = -0.0
+    W[0, 65] = 0.5
+    codes, a = oracle.quantize(W)
+    assert a[0] == 0 and a[1] == 0.5
+    assert np.all(codes[:64] == 7)        # all-zero block -> the exact-zero row
+    assert codes[64] == 7                 # -0.0 -> zero row
+    assert codes[65] == 15                # +absmax -> +1 row
+    Wd = oracle.dequantize(oracle.pack(codes), a, W.shape)
+    assert np.all(Wd[0, :64] == 0) and not np.signbit(Wd[0, 64])
+
+
+def test_absmax_element_maps_to_table_ends():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((8, 256)) * 0.02).astype(np.float32)
+    codes, a = oracle.quantize(W)
+    blk = W.reshape(-1, 64)
+    c = codes.reshape(-1, 64)
+    for b in range(blk.shape[0]):
+        i = int(np.argmax(np.abs(blk[b])))
+        assert c[b, i] == (15 if blk[b, i] > 0 else 0)
+
+
+def test_permutation_and_power_of_two_scaling():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((2, 64)) * 0.02).astype(np.float32)
+    codes, a = oracle.quantize(W)
+    perm = rng.permutation(64)
+    codes_p, a_p = oracle.quantize(W[:, perm])
+    assert np.array_equal(codes_p.reshape(2, 64), codes.reshape(2, 64)[:, perm])
+    assert np.array_equal(a_p, a)
+    codes_s, a_s = oracle.quantize(W * np.float32(2.0 ** -5))
+    assert np.array_equal(codes_s, codes)
+    assert np.array_equal(a_s, a * np.float32(2.0 ** -5))
+
+
+def test_outlier_damage_stays_in_its_block():
+    """'Keeping groups small keeps an outlier's damage inside its own group.'"""
+    rng = np.random.default_rng(13)
+    W = (rng.standard_normal((4, 256)) * 0.02).astype(np.float32)
+    W2 = W.copy()
+    W2[1, 70] = 3.0                       # block index (256 + 70) // 64 = 5
+    c1, a1 = oracle.quantize(W)
+    c2, a2 = oracle.quantize(W2)
+    diff_blocks = np.unique(np.nonzero(c1 != c2)[0] // 64)
+    assert list(diff_blocks) == [5]
+    assert list(np.nonzero(a1 != a2)[0]) == [5]
+    # the outlier block's ordinary weights collapse onto the middle rows
+    assert np.all(np.isin(np.delete(c2.reshape(-1, 64)[5], 6), [6, 7, 8]))
+
+
+def test_nonfinite_rejected():
+    W = np.zeros((1, 64), dtype=np.float32)
+    W[0, 3] = np.nan
+    with pytest.raises(ValueError):
+        oracle.quantize(W)
+    W[0, 3] = np.inf
+    with pytest.raises(ValueError):
+        oracle.quantize(W)
+
+
+def test_pack_nibble_order_and_roundtrip():
+    codes = np.array([1, 2, 3, 4, 15, 0], dtype=np.uint8)
+    p = oracle.pack(codes)
+    assert list(p) == [0x12, 0x34, 0xF0]
+    rng = np.random.default_rng(1)
+    c = rng.integers(0, 16, 1000).astype(np.uint8)
+    assert np.array_equal(oracle.unpack(oracle.pack(c)), c)
+    assert oracle.pack(c).size == 500
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding vs torch
+# ---------------------------------------------------------------------------
+
+def test_round_bf16_matches_torch():
+    rng = np.random.default_rng(2)
+    x = np.concatenate([
+        rng.standard_normal(100000).astype(np.float32) * 0.02,
+        rng.standard_normal(1000).astype(np.float32) * 1e-38,
+        # exact ties: low 16 bits == 0x8000, both parities of the kept part
+        (np.arange(1000, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
+        np.array([0.0, -0.0, 1.0, -1.0], dtype=np.float32),
+    ])
+    want = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    got = oracle.round_bf16(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# Double quantisation
+# ---------------------------------------------------------------------------
+
+def test_dq_mean_exact():
+    """mu against an exact rational mean (tiny) and an fp64 running sum (large)."""
+    rng = np.random.default_rng(4)
+    a = np.abs(rng.standard_normal(1000).astype(np.float32)) * np.float32(0.05)
+    exact = sum(Fraction(float(v)) for v in a) / len(a)
+    mu = oracle.dq_mean(a)
+    # RN32 of RN64(sum)/n: within half an fp32 ulp of the exact mean plus 2^-52 relative
+    assert abs(Fraction(float(mu)) - exact) <= Fraction(float(np.spacing(mu))) / 2 + exact * Fraction(1, 2 ** 51)
+    big = np.abs(rng.standard_normal(200000).astype(np.float32))
+    s = 0.0
+    for v in big.astype(np.float64):
+        s += v
+    assert oracle.dq_mean(big) == np.float32(s / big.size)
+
+
+def test_double_quantize_properties():
+    rng = np.random.default_rng(6)
+    a = np.abs(rng.standard_normal(1000).astype(np.float32)) * np.float32(0.05)   # 3 full groups + 1 partial
+    q, s, mu = oracle.double_quantize(a)
+    assert q.dtype == np.int8 and s.shape == (4,)
+    d = (a - mu).astype(np.float32)
+    for g in range(4):
+        dg = d[g * 256:(g + 1) * 256]
+        assert s[g] == np.abs(dg).max()
+        qg = q[g * 256:(g + 1) * 256]
+        assert np.abs(qg).max() == 127
+        assert qg[int(np.argmax(np.abs(dg)))] == (127 if dg[np.argmax(np.abs(dg))] > 0 else -127)
+    ah = oracle.dq_absmax(q, s, mu)
+    sg = np.repeat(s, 256)[:a.size]
+    bound = sg / 254 + 4 * np.spacing(np.maximum(np.abs(a), np.abs(ah)))
+    assert np.all(np.abs(ah.astype(np.float64) - a) <= bound)
+
+
+def test_double_quantize_constant_group():
+    a = np.full(300, 0.25, dtype=np.float32)
+    q, s, mu = oracle.double_quantize(a)
+    assert mu == np.float32(0.25)
+    assert np.all(s == 0) and np.all(q == 0)
+    assert np.all(oracle.dq_absmax(q, s, mu) == np.float32(0.25))
+
+
+def test_storage_closed_forms(golden):
+    g = golden
+    n = 4096 * 4096
+    assert oracle.stored_bits_per_param(n, double_quant=False) - 4 == g["fp32_scale_bits"]
+    assert (oracle.stored_bits_per_param(n, double_quant=False) - 4) / 4 == g["fp32_scale_surcharge"]
+    bits = oracle.stored_bits_per_param(n)
+    assert bits == 4 + 8 / 64 + 32 / 16384 + 32 / n
+    assert 8 / 64 == g["dq_scale_bits"]
+    assert 32 / 16384 == pytest.approx(g["dq_group_bits"], abs=5e-4)
+    assert bits == pytest.approx(g["total_bits"], abs=0.005)
+    assert g["total_bits"] / 8 == g["bytes_per_param"]
+    saving = oracle.stored_bits_per_param(n, double_quant=False) - bits + 32 / n
+    assert saving == 0.373046875
+    assert saving == pytest.approx(g["dq_saving_bits"], abs=0.005)
+    assert saving < g["dq_saving_bits_upper"]
+    assert g["model_7b_params"] * g["bytes_per_param"] / 1e9 == pytest.approx(g["model_7b_nf4_gb"], abs=0.05)
+    assert g["model_7b_params"] * 2 / 1e9 == pytest.approx(g["model_7b_bf16_gb"], abs=0.05)
+    # N x b / 8
+    assert g["model_13b_params"] * 16 / 8 / 1e9 == g["model_13b_fp16_gb"]
+    assert g["model_13b_params"] * 4 / 8 / 1e9 == g["model_13b_4bit_gb"]
+    # rank-16 adapter on a 4096 x 4096 projection: r*(d+k) = 2rd
+    r, d = 16, 4096
+    assert r * (d + d) == 2 * r * d == 131072
+    assert r * (d + d) == pytest.approx(g["lora_rank16_4096_params"], rel=0.01)
+    assert d * d == pytest.approx(g["base_4096_params"], rel=0.01)
+
+
+# ---------------------------------------------------------------------------
+# Dequantise
+# ---------------------------------------------------------------------------
+
+def test_dequantize_invariants():
+    rng = np.random.default_rng(8)
+    W = (rng.standard_normal((16, 512)) * 0.02).astype(np.float32)
+    codes, a = oracle.quantize(W)
+    q, s, mu = oracle.double_quantize(a)
+    ah = oracle.dq_absmax(q, s, mu)
+    for aa in (a, ah):
+        Wd = oracle.dequantize(oracle.pack(codes), aa, W.shape)
+        blk = Wd.reshape(-1, 64)
+        wb = W.reshape(-1, 64)
+        for b in range(blk.shape[0]):
+            assert len(np.unique(blk[b])) <= 16
+            i = int(np.argmax(np.abs(wb[b])))
+            want = oracle.round_bf16(np.array([aa[b]], np.float32))[0]
+            assert blk[b, i] == (want if wb[b, i] > 0 else -want)
+        # values are bf16-representable
+        assert np.array_equal(oracle.round_bf16(Wd), Wd)
+        # re-quantising the dequantised weights reproduces the codes (soft
+        # invariant; holds on this seed)
+        c2, _ = oracle.quantize(Wd)
+        assert np.mean(c2 == codes) > 0.999
+
+
+def test_dequantize_matches_table_times_scale_closed_form():
+    """Each element equals RNbf16(q[code] * a^): check with torch's bf16 cast."""
+    rng = np.random.default_rng(10)
+    W = (rng.standard_normal((4, 128)) * 0.02).astype(np.float32)
+    codes, a = oracle.quantize(W)
+    Wd = oracle.dequantize(oracle.pack(codes), a, W.shape)
+    q = oracle.nf4_table()
+    ref = torch.from_numpy((q[codes] * np.repeat(a, 64)).astype(np.float32)).to(torch.bfloat16).float()
+    assert np.array_equal(Wd.reshape(-1), ref.numpy())
+
+
+# ---------------------------------------------------------------------------
+# Linear layer vs torch.autograd (fp64)
+# ---------------------------------------------------------------------------
+
+def test_linear_fwd_bwd_vs_autograd():
+    torch.manual_seed(0)
+    M, N, K, r, alpha = 5, 7, 64, 4, 8.0
+    X = torch.randn(M, K, dtype=torch.float64, requires_grad=True)
+    W = torch.randn(N, K, dtype=torch.float64)
+    A = torch.randn(r, K, dtype=torch.float64, requires_grad=True)
+    B = torch.randn(N, r, dtype=torch.float64, requires_grad=True)
+    dY = torch.randn(M, N, dtype=torch.float64)
+    # W' = W + s B A (LoRA page), applied as a Linear: Y = X W'^T
+    Y = torch.nn.functional.linear(X, W + (alpha / r) * (B @ A))
+    Y.backward(dY)
+    Yo, T = oracle.linear_fwd(X.detach().numpy(), W.numpy(), A.detach().numpy(),
+                              B.detach().numpy(), alpha, r)
+    dX, dA, dB = oracle.linear_bwd(X.detach().numpy(), dY.numpy(), W.numpy(),
+                                   A.detach().numpy(), B.detach().numpy(), alpha, r)
+    assert np.allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dX, X.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dA, A.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dB, B.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_special_cases():
+    rng = np.random.default_rng(12)
+    M, N, K, r = 6, 8, 64, 4
+    X = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K))
+    A = rng.standard_normal((r, K))
+    Y, _ = oracle.linear_fwd(X, W, A, np.zeros((N, r)), 8.0, r)
+    assert np.allclose(Y, torch.from_numpy(X) @ torch.from_numpy(W).T, rtol=1e-13)
+    # one-hot token rows with A = 0 read out columns of W exactly
+    E = np.eye(K)[:M]
+    Y, _ = oracle.linear_fwd(E, W, np.zeros((r, K)), rng.standard_normal((N, r)), 8.0, r)
+    assert np.array_equal(Y, W[:, :M].T)
+    # finite difference on one A entry
+    B = rng.standard_normal((N, r))
+    dY = rng.standard_normal((M, N))
+    _, dA, _ = oracle.linear_bwd(X, dY, W, A, B, 8.0, r)
+    eps = 1e-6
+    A2 = A.copy()
+    A2[1, 3] += eps
+    Y1, _ = oracle.linear_fwd(X, W, A, B, 8.0, r)
+    Y2, _ = oracle.linear_fwd(X, W, A2, B, 8.0, r)
+    fd = np.sum(dY * (Y2 - Y1)) / eps
+    assert fd == pytest.approx(dA[1, 3], rel=1e-5)
+
+
+def test_bf16_in_fp64_products_are_exact():
+    """The oracle's fp64 matmul of bf16 inputs: each product is exact (8+8
+    significant bits), so for K <= 2^20 the fp64 sum error is tiny relative to
+    the 1e-2 bar.  Check one dot product against exact rationals."""
+    rng = np.random.default_rng(14)
+    x = oracle.round_bf16(rng.standard_normal(4096).astype(np.float32)).astype(np.float64)
+    w = oracle.round_bf16((rng.standard_normal(4096) * 0.02).astype(np.float32)).astype(np.float64)
+    exact = sum(Fraction(a) * Fraction(b) for a, b in zip(x, w))
+    got = float(np.dot(x, w))
+    assert abs(Fraction(got) - exact) <= Fraction(1, 2 ** 40) * max(1, abs(exact))
+    assert math.isfinite(got)
