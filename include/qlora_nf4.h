@@ -1,0 +1,200 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: blockwise NF4 quantisation, double
+ * quantisation and the QLoRA linear layer (forward, input/adapter backward)
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web pages, cited by title and section):
+ *   [QE]  "QLoRA Explained: A 4-Bit Base, NF4, and What It Really Costs"
+ *         (skillsuites.com)
+ *   [LQ]  "LoRA vs QLoRA: Efficient Fine-Tuning Explained" (masterainow.com)
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates nothing: scratch space is a caller-provided workspace
+ *    whose size comes from qlora_workspace_bytes().
+ *  - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *    stream).  Returning QLORA_OK means "validated and enqueued".
+ *  - Arguments are validated synchronously before anything is enqueued; on a
+ *    validation error nothing is launched and the status is returned.
+ *  - Errors detected on the device (a non-finite weight, a bounded wait that
+ *    ran out) set a sticky per-device status word; qlora_check_status()
+ *    synchronises the stream, returns that word and clears it.
+ *  - Matrices are row-major with dense rows.  bf16 is IEEE bfloat16 passed
+ *    as 16-bit storage (uint16_t / torch.bfloat16).
+ *  - Every device pointer must be 16-byte aligned.
+ *  - There is no CPU fallback: without a usable sm_100 device every compute
+ *    entry point returns QLORA_ERR_CUDA or QLORA_ERR_UNSUPPORTED.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* qlora_stream_t;
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, bad rank/alpha      */
+  QLORA_ERR_SHAPE = 2,         /* a dimension violates a stated constraint    */
+  QLORA_ERR_ALIGN = 3,         /* a pointer is not 16-byte aligned            */
+  QLORA_ERR_NONFINITE = 4,     /* device: NaN/Inf weight met while quantising */
+  QLORA_ERR_TIMEOUT = 5,       /* device: a bounded pipeline wait gave up     */
+  QLORA_ERR_CUDA = 6,          /* a CUDA runtime/driver call failed           */
+  QLORA_ERR_UNSUPPORTED = 7,   /* no sm_100 device, or a mode not built       */
+  QLORA_ERR_WORKSPACE = 8      /* workspace null or smaller than required     */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* Operation ids for qlora_workspace_bytes(). */
+typedef enum {
+  QLORA_OP_DOUBLE_QUANT = 0,
+  QLORA_OP_FWD = 1,
+  QLORA_OP_BWD = 2
+} qlora_op;
+
+/*
+ * A quantised frozen weight W[rows, cols] (rows = N output features,
+ * cols = K input features).  [QE] "Why the groups are small": one scale per
+ * block of 64 consecutive weights of the row-major flattening (cols % 64 == 0,
+ * so blocks never straddle rows).  [QE] "Shrink the scale factors too": with
+ * double quantisation the block scales are int8 in groups of 256 with one
+ * fp32 scale per group, plus one fp32 mean offset per tensor.
+ *
+ *   packed   [rows*cols/2]  two codes per byte, element 2j in the HIGH nibble
+ *   absmax   [rows*cols/64] fp32 block scales      (used when double_quant == 0)
+ *   qabsmax  [rows*cols/64] int8 block-scale codes (used when double_quant == 1)
+ *   dq_scale [ceil(rows*cols/64/256)] fp32 group scales (double_quant == 1)
+ *   dq_mean  [1] fp32 per-tensor mean offset, device     (double_quant == 1)
+ *
+ * Dequantised value of element i in block b (code c, table q):
+ *   a^ = absmax[b]                                              (no DQ)
+ *   a^ = RN32(RN32(RN32(qabsmax[b]/127) * dq_scale[b/256]) + dq_mean) (DQ)
+ *   w' = RNbf16(RN32(q[c] * a^))
+ */
+typedef struct {
+  const uint8_t* packed;
+  int64_t rows;
+  int64_t cols;
+  int32_t blocksize;      /* must be 64  */
+  int32_t double_quant;   /* 0 or 1      */
+  const float* absmax;
+  const int8_t* qabsmax;
+  const float* dq_scale;
+  const float* dq_mean;
+  int32_t dq_blocksize;   /* must be 256 */
+} nf4_weight;
+
+/* ---- host-only queries (no GPU needed) -------------------------------- */
+
+/* The library's 16-entry NF4 table and its 15 decision thresholds, computed
+ * on the host at load time ([QE] "Put the rows where the weights are",
+ * "That is NF4": normal quantiles normalised to [-1, 1], exact zero; ties
+ * between two rows go to the higher row, [QE] "The two failures ...").
+ * Writes 16 (resp. 15) floats.  Returns QLORA_OK or QLORA_ERR_INVALID_ARG. */
+int nf4_code_table(float* table16);
+int nf4_code_thresholds(float* thresholds15);
+
+/* Bytes of caller workspace needed by an operation (0 if none).
+ *   QLORA_OP_DOUBLE_QUANT: M, K, r ignored; N = number of absmax values.
+ *   QLORA_OP_FWD / QLORA_OP_BWD: layer with M tokens, weight N x K, rank r. */
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
+
+/* Human-readable name of a status code (static string). */
+const char* qlora_status_string(int status);
+
+/* ABI version of this header (major*100 + minor). */
+int qlora_abi_version(void);
+
+/* ---- device entry points ---------------------------------------------- */
+
+/*
+ * Blockwise NF4 quantisation ([QE] "The table, and the number that stretches
+ * it", steps 1-3; "Why the groups are small").
+ *   W       device [rows, cols], fp32 or bf16 (dtype)
+ *   packed  device out [rows*cols/2]
+ *   absmax  device out [rows*cols/64] fp32
+ * Per block: a = max|w| (exact); x = RN32(w / a) (IEEE division); code =
+ * index of the nearest table row, ties to the higher row; a zero block gives
+ * code 7 (the exact zero) everywhere.  Constraints: rows >= 1, cols >= 64,
+ * cols % 64 == 0, blocksize == 64.  A NaN/Inf weight sets
+ * QLORA_ERR_NONFINITE in the device status word (outputs then undefined).
+ */
+int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols,
+                 int blocksize, uint8_t* packed, float* absmax,
+                 qlora_stream_t stream);
+
+/*
+ * Double quantisation of the block scales ([QE] "Shrink the scale factors
+ * too").  mean = RN32(RN64(exact sum of absmax) / n) (one per tensor);
+ * d = RN32(a - mean); s_g = max|d| over each group of 256 (the last group may
+ * be partial); c = round-half-even(RN32(RN32(d / s_g) * 127)), 0 if s_g == 0.
+ *   absmax   device [n_absmax] fp32, finite and >= 0
+ *   qabsmax  device out [n_absmax] int8
+ *   dq_scale device out [ceil(n_absmax/256)] fp32
+ *   dq_mean  device out [1] fp32
+ *   ws       device workspace of qlora_workspace_bytes(QLORA_OP_DOUBLE_QUANT, ..)
+ * The mean is bit-identical for any launch order (exact integer sum).
+ */
+int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
+                        int8_t* qabsmax, float* dq_scale, float* dq_mean,
+                        void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Dequantise to bf16 ([QE] worked example step 4; "That is NF4": every
+ * matmul runs on values expanded back to bf16).
+ *   W_out device out [rows, cols] bf16,  w' = RNbf16(RN32(q[code] * a^)).
+ */
+int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream);
+
+/*
+ * QLoRA linear forward ([LQ] "How LoRA Works": W' = W + (alpha/r) B A;
+ * [QE] "Why the expansion cannot be skipped": codes -> table -> scale ->
+ * bf16 on chip -> tensor core):
+ *   Y = X deq(W)^T + s (X A^T) B^T,   s = alpha / r,  fp32 accumulation.
+ *   X  device [M, K] bf16      A device [r, K] bf16    B device [N, r] bf16
+ *   Y  device out [M, N] bf16
+ *   T_save device out [M, r] bf16 = RNbf16(X A^T), or NULL
+ *   ws device workspace of qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r)
+ * Constraints: M >= 1, N % 8 == 0, K % 64 == 0, r in {8,16,32,64,128},
+ * alpha finite.  M <= 16 runs the decode (GEMV) kernel, larger M the fused
+ * dequantise-in-mainloop tensor-core GEMM.
+ */
+int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M,
+                     const void* A, const void* B, int r, float alpha,
+                     void* Y, void* T_save, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream);
+
+/*
+ * QLoRA linear backward ([LQ] "How QLoRA Works": the frozen base gets no
+ * gradient; only the adapters do).  With U = dY B:
+ *   dX = dY deq(W) + s U A      [M, K] bf16
+ *   dA = s U^T X                [r, K] bf16
+ *   dB = s dY^T (X A^T)         [N, r] bf16
+ *   T  device [M, r] bf16 = X A^T saved by the forward, or NULL to recompute
+ * Same constraints as the forward; reductions over M are fixed-order
+ * (deterministic).
+ */
+int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY,
+                     int64_t M, const void* A, const void* B, int r,
+                     float alpha, const void* T, void* dX, void* dA, void* dB,
+                     void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Synchronise `stream`, return the sticky device status word (QLORA_OK if
+ * no device-side error was recorded since the last call) and clear it.
+ */
+int qlora_check_status(qlora_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,97 @@
+"""ctypes loader for libqlora_nf4.so: argument marshalling only.
+
+The C ABI is declared in include/qlora_nf4.h.  This module maps each entry
+point to a Python callable of the same name taking plain integers (device
+addresses), sizes and stream handles.  It never computes anything itself and
+has no fallback: if the library is missing, importing it raises.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlora_nf4.so")
+
+QLORA_OK = 0
+QLORA_ERR_INVALID_ARG = 1
+QLORA_ERR_SHAPE = 2
+QLORA_ERR_ALIGN = 3
+QLORA_ERR_NONFINITE = 4
+QLORA_ERR_TIMEOUT = 5
+QLORA_ERR_CUDA = 6
+QLORA_ERR_UNSUPPORTED = 7
+QLORA_ERR_WORKSPACE = 8
+
+QLORA_F32 = 0
+QLORA_BF16 = 1
+
+QLORA_OP_DOUBLE_QUANT = 0
+QLORA_OP_FWD = 1
+QLORA_OP_BWD = 2
+
+# Every symbol the header declares, with (restype, argtypes).
+_vp, _i64, _i32, _f32, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
+
+
+class NF4Weight(C.Structure):
+    """Mirror of `nf4_weight` in include/qlora_nf4.h."""
+    _fields_ = [
+        ("packed", _vp),
+        ("rows", _i64),
+        ("cols", _i64),
+        ("blocksize", C.c_int32),
+        ("double_quant", C.c_int32),
+        ("absmax", _vp),
+        ("qabsmax", _vp),
+        ("dq_scale", _vp),
+        ("dq_mean", _vp),
+        ("dq_blocksize", C.c_int32),
+    ]
+
+
+SIGNATURES = {
+    "qlora_abi_version": (_i32, []),
+    "qlora_status_string": (C.c_char_p, [_i32]),
+    "nf4_code_table": (_i32, [C.POINTER(C.c_float)]),
+    "nf4_code_thresholds": (_i32, [C.POINTER(C.c_float)]),
+    "qlora_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
+    "nf4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "nf4_double_quantize": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nf4_dequantize": (_i32, [C.POINTER(NF4Weight), _vp, _vp]),
+    "qlora_linear_fwd": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
+                                _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i64, _vp, _vp, _i32, _f32,
+                                _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_check_status": (_i32, [_vp]),
+}
+
+_lib = None
+
+
+def load() -> C.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m qlora_linear_layers_b200.build`")
+        lib = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = load().qlora_status_string(code).decode()
+        super().__init__(f"{where}: {msg} (status {code})")
+
+
+def check(code: int, where: str) -> None:
+    if code != QLORA_OK:
+        raise QLoraError(code, where)

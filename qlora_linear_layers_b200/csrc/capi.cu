@@ -1,0 +1,213 @@
+// C ABI of libqlora_nf4.so: argument validation, workspace sizing, dispatch
+// to the sm_100a kernels, and the sticky device status word.
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qnf4 {
+
+// One status word per device (each device context has its own copy).
+static __device__ int g_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int major = 0, minor = 0;
+  int* status = nullptr;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Returns QLORA_OK and fills `info` for the current device, or an error if
+// there is no usable sm_100 device.
+int current_device(DeviceInfo** info) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_CUDA; }
+    d.sms = p.multiProcessorCount;
+    d.major = p.major;
+    d.minor = p.minor;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_CUDA; }
+    d.status = static_cast<int*>(ptr);
+    d.ready = true;
+  }
+  if (d.major != 10) return QLORA_ERR_UNSUPPORTED;   // sm_100 family only
+  *info = &d;
+  return QLORA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+int check_weight(const nf4_weight* w) {
+  if (!w || !w->packed) return QLORA_ERR_INVALID_ARG;
+  if (w->blocksize != 64) return QLORA_ERR_UNSUPPORTED;
+  if (w->rows < 1 || w->cols < 64 || w->cols % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
+  if (w->double_quant) {
+    if (w->dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
+    if (!w->qabsmax || !w->dq_scale || !w->dq_mean) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->qabsmax) || !aligned16(w->dq_scale) || !aligned16(w->dq_mean))
+      return QLORA_ERR_ALIGN;
+  } else {
+    if (!w->absmax) return QLORA_ERR_INVALID_ARG;
+    if (!aligned16(w->absmax)) return QLORA_ERR_ALIGN;
+  }
+  return QLORA_OK;
+}
+
+}  // namespace
+
+int* device_status_ptr() {
+  DeviceInfo* d = nullptr;
+  return current_device(&d) == QLORA_OK ? d->status : nullptr;
+}
+
+}  // namespace qnf4
+
+using namespace qnf4;
+
+extern "C" {
+
+int qlora_abi_version(void) { return 100; }
+
+const char* qlora_status_string(int s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_SHAPE: return "shape violates a constraint";
+    case QLORA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case QLORA_ERR_NONFINITE: return "non-finite value met on the device";
+    case QLORA_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case QLORA_ERR_CUDA: return "CUDA call failed";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported device or mode";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int nf4_code_table(float* table16) {
+  if (!table16) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(table16, host_tables().q, 16 * sizeof(float));
+  return QLORA_OK;
+}
+
+int nf4_code_thresholds(float* thresholds15) {
+  if (!thresholds15) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(thresholds15, host_tables().t, 15 * sizeof(float));
+  return QLORA_OK;
+}
+
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
+  (void)M; (void)N; (void)K; (void)r;
+  switch (op) {
+    case QLORA_OP_DOUBLE_QUANT: return 256 * sizeof(unsigned long long);
+    default: return 0;
+  }
+}
+
+int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols, int blocksize,
+                 uint8_t* packed, float* absmax, qlora_stream_t stream) {
+  if (!W || !packed || !absmax) return QLORA_ERR_INVALID_ARG;
+  if (dtype != QLORA_F32 && dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (blocksize != 64) return QLORA_ERR_UNSUPPORTED;
+  if (rows < 1 || cols < 64 || cols % 64) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(absmax)) return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  int st = current_device(&d);
+  if (st) return st;
+  launch_quantize(W, dtype, rows * cols, packed, absmax, d->status, (cudaStream_t)stream, d->sms);
+  return launch_status();
+}
+
+int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize, int8_t* qabsmax,
+                        float* dq_scale, float* dq_mean, void* ws, size_t ws_bytes,
+                        qlora_stream_t stream) {
+  if (!absmax || !qabsmax || !dq_scale || !dq_mean) return QLORA_ERR_INVALID_ARG;
+  if (dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
+  if (n_absmax < 1) return QLORA_ERR_SHAPE;
+  if (!ws || ws_bytes < qlora_workspace_bytes(QLORA_OP_DOUBLE_QUANT, 0, n_absmax, 0, 0))
+    return QLORA_ERR_WORKSPACE;
+  if (!aligned16(absmax) || !aligned16(qabsmax) || !aligned16(dq_scale) || !aligned16(dq_mean) ||
+      !aligned16(ws))
+    return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  int st = current_device(&d);
+  if (st) return st;
+  launch_double_quantize(absmax, n_absmax, qabsmax, dq_scale, dq_mean,
+                         static_cast<unsigned long long*>(ws), d->status, (cudaStream_t)stream,
+                         d->sms);
+  return launch_status();
+}
+
+int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
+  int st = check_weight(w);
+  if (st) return st;
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  st = current_device(&d);
+  if (st) return st;
+  launch_dequantize(w, W_out, (cudaStream_t)stream, d->sms);
+  return launch_status();
+}
+
+int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
+                     int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
+  (void)w; (void)X; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)Y; (void)T_save;
+  (void)ws; (void)ws_bytes; (void)stream;
+  return QLORA_ERR_UNSUPPORTED;
+}
+
+int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
+                     const void* B, int r, float alpha, const void* T, void* dX, void* dA,
+                     void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  (void)w; (void)X; (void)dY; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)T;
+  (void)dX; (void)dA; (void)dB; (void)ws; (void)ws_bytes; (void)stream;
+  return QLORA_ERR_UNSUPPORTED;
+}
+
+int qlora_check_status(qlora_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  DeviceInfo* d = nullptr;
+  int st = current_device(&d);
+  if (st) return st;
+  int v = 0;
+  if (cudaMemcpy(&v, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(d->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,20 @@
+// Launchers shared between the C-ABI layer (capi.cu) and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora_nf4.h"
+
+namespace qnf4 {
+
+void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
+                     int* status, cudaStream_t s, int num_sms);
+
+void launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
+                            float* dq_mean, unsigned long long* hist, int* status,
+                            cudaStream_t s, int num_sms);
+
+void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms);
+
+}  // namespace qnf4

@@ -1,0 +1,95 @@
+// Host-side construction of the NF4 table and its decision thresholds.
+//
+// Page "QLoRA Explained", sections "Put the rows where the weights are" and
+// "That is NF4": the 16 rows sit at quantiles of a standard normal, are
+// computed once (not from the model) and include an exact zero; the table is
+// normalised onto [-1, 1] so that a block's absmax stretches it onto the
+// weights.  The page gives no construction for the exact zero; this library
+// uses 8 positive levels, the zero and 7 negative levels:
+//   delta = (1/30 + 1/32) / 2, top = 1 - delta
+//   positive: Phi^-1 at 8 probabilities spaced evenly from top towards 1/2
+//             (9 points including 1/2, which is dropped)
+//   negative: -Phi^-1 at 7 such probabilities (8 points, 1/2 dropped)
+//   divide by Phi^-1(top) so the ends are exactly -1 and +1; round to fp32.
+// Phi^-1 is found by bisection on Phi(z) = erfc(-z / sqrt 2) / 2 in double
+// precision, which converges to the double nearest the root (well inside the
+// fp32 rounding of the final values).
+//
+// Thresholds: a value x goes to the nearest row, a tie to the higher row
+// (page "QLoRA Explained", section "The two failures that motivate the next
+// section": 0, exactly between two rows, comes back as the upper one).  For
+// rows q_j < q_{j+1} the decision point is their exact midpoint (exact in
+// double); for an fp32 x, "x >= midpoint" equals "x >= T_j" with T_j the
+// smallest float not below the midpoint.
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+static double normal_cdf(double z) { return 0.5 * std::erfc(-z / std::sqrt(2.0)); }
+
+static double normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0;
+  for (int i = 0; i < 2000 && lo < hi; ++i) {
+    double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (normal_cdf(mid) < p) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+static Nf4Tables build_tables() {
+  Nf4Tables tb{};
+  const double delta = 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+  const double top = 1.0 - delta;
+  std::vector<double> lv;
+  for (int i = 0; i < 8; ++i) lv.push_back(normal_quantile(top + (0.5 - top) * i / 8.0));
+  for (int i = 0; i < 7; ++i) lv.push_back(-normal_quantile(top + (0.5 - top) * i / 7.0));
+  lv.push_back(0.0);
+  std::sort(lv.begin(), lv.end());
+  double mx = 0.0;
+  for (double v : lv) mx = std::max(mx, std::fabs(v));
+  for (int i = 0; i < 16; ++i) tb.q[i] = (float)(lv[i] / mx);
+
+  for (int j = 0; j < 15; ++j) {
+    double m = ((double)tb.q[j] + (double)tb.q[j + 1]) * 0.5;   // exact
+    float t = (float)m;
+    if ((double)t < m) t = std::nextafter(t, INFINITY);
+    tb.t[j] = t;
+  }
+
+  // Bucket table for the quantise kernel's code search.  Every threshold
+  // must sit well away from a bucket edge so that the rounding in the
+  // bucket index (x + 1) * 16 can never put x on the wrong side of an edge
+  // that a threshold shares.
+  for (int b = 0; b < 32; ++b) {
+    double lo = -1.0 + b / 16.0, hi = lo + 1.0 / 16.0;
+    int base = 0;
+    float thr = INFINITY;
+    for (int j = 0; j < 15; ++j) {
+      if ((double)tb.t[j] < lo) ++base;
+      else if ((double)tb.t[j] < hi) {
+        if (thr != INFINITY) { std::fprintf(stderr, "qlora_nf4: two thresholds in a bucket\n"); std::abort(); }
+        thr = tb.t[j];
+      }
+      double edge_gap = std::min(std::fabs((double)tb.t[j] - lo), std::fabs((double)tb.t[j] - hi));
+      if (edge_gap < 1e-4) { std::fprintf(stderr, "qlora_nf4: threshold too near a bucket edge\n"); std::abort(); }
+    }
+    tb.bucket_base[b] = (uint8_t)base;
+    tb.bucket_thr[b] = thr;
+  }
+  return tb;
+}
+
+const Nf4Tables& host_tables() {
+  static const Nf4Tables tb = build_tables();
+  return tb;
+}
+
+}  // namespace qnf4

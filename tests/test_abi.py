@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI (no GPU, no compute calls).
+
+* the library loads and exports every function include/qlora_nf4.h declares;
+* its host-computed NF4 table and thresholds equal the oracle's bit for bit
+  (two independent constructions: the library bisects libm's erfc, the
+  oracle uses Python's statistics.NormalDist);
+* argument validation rejects bad calls before touching a device.
+"""
+
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from qlora_linear_layers_b200 import _lib
+from qlora_linear_layers_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "qlora_nf4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "sizeof")))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES)
+    assert lib.qlora_abi_version() == 100
+
+
+def test_library_table_matches_oracle(lib):
+    buf = (C.c_float * 16)()
+    assert lib.nf4_code_table(buf) == 0
+    got = np.frombuffer(buf, dtype=np.float32)
+    want = oracle.nf4_table()
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    tb = (C.c_float * 15)()
+    assert lib.nf4_code_thresholds(tb) == 0
+    assert np.array_equal(np.frombuffer(tb, dtype=np.float32), oracle.thresholds(want))
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        assert lib.qlora_status_string(code)
+    assert lib.qlora_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    assert lib.qlora_workspace_bytes(_lib.QLORA_OP_DOUBLE_QUANT, 0, 1000, 0, 0) == 2048
+
+
+def test_validation_before_any_device_call(lib):
+    # Null pointers, bad shapes, misalignment: rejected synchronously.  The
+    # fake addresses below are never dereferenced (validation fails first).
+    fake = 1 << 20
+    assert lib.nf4_quantize(None, 1, 64, 64, 64, fake, fake, None) == _lib.QLORA_ERR_INVALID_ARG
+    assert lib.nf4_quantize(fake, 7, 64, 64, 64, fake, fake, None) == _lib.QLORA_ERR_INVALID_ARG
+    assert lib.nf4_quantize(fake, 1, 64, 64, 32, fake, fake, None) == _lib.QLORA_ERR_UNSUPPORTED
+    assert lib.nf4_quantize(fake, 1, 64, 96, 64, fake, fake, None) == _lib.QLORA_ERR_SHAPE
+    assert lib.nf4_quantize(fake, 1, 0, 64, 64, fake, fake, None) == _lib.QLORA_ERR_SHAPE
+    assert lib.nf4_quantize(fake + 2, 1, 64, 64, 64, fake, fake, None) == _lib.QLORA_ERR_ALIGN
+    assert lib.nf4_double_quantize(fake, 100, 128, fake, fake, fake, fake, 4096, None) == \
+        _lib.QLORA_ERR_UNSUPPORTED
+    assert lib.nf4_double_quantize(fake, 100, 256, fake, fake, fake, None, 0, None) == \
+        _lib.QLORA_ERR_WORKSPACE
+    assert lib.nf4_double_quantize(fake, 100, 256, fake, fake, fake, fake, 16, None) == \
+        _lib.QLORA_ERR_WORKSPACE
+    w = _lib.NF4Weight(packed=fake, rows=64, cols=64, blocksize=64, double_quant=1,
+                       absmax=None, qabsmax=None, dq_scale=fake, dq_mean=fake, dq_blocksize=256)
+    assert lib.nf4_dequantize(C.byref(w), fake, None) == _lib.QLORA_ERR_INVALID_ARG
+    w.qabsmax = fake
+    w.cols = 100
+    assert lib.nf4_dequantize(C.byref(w), fake, None) == _lib.QLORA_ERR_SHAPE
