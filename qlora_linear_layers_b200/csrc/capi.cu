@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "gemm.h"
 
 namespace qnf4 {
 
@@ -55,6 +56,25 @@ int current_device(DeviceInfo** info) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool valid_rank(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+int padded_rank(int r) { return r <= 64 ? 64 : 128; }
+
+// Forward workspace: sT_pad [M, RP] bf16, then Bpad [N, RP] bf16 when r < RP.
+struct FwdWs {
+  size_t sT, Bpad, total;
+};
+FwdWs fwd_ws(int64_t M, int64_t N, int r) {
+  FwdWs w{};
+  const int RP = padded_rank(r);
+  w.sT = 0;
+  w.Bpad = align256((size_t)M * RP * 2);
+  w.total = w.Bpad + (r < RP ? align256((size_t)N * RP * 2) : 0);
+  return w;
+}
 
 int launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -121,9 +141,12 @@ int nf4_code_thresholds(float* thresholds15) {
 }
 
 size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
-  (void)M; (void)N; (void)K; (void)r;
+  (void)K;
   switch (op) {
     case QLORA_OP_DOUBLE_QUANT: return 256 * sizeof(unsigned long long);
+    case QLORA_OP_FWD:
+      if (M < 1 || N < 1 || !valid_rank(r)) return 0;
+      return fwd_ws(M, N, r).total;
     default: return 0;
   }
 }
@@ -177,9 +200,47 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
 int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
                      int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {
-  (void)w; (void)X; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)Y; (void)T_save;
-  (void)ws; (void)ws_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  int st = check_weight(w);
+  if (st) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!valid_rank(r) || !(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return QLORA_ERR_INVALID_ARG;
+  const int64_t N = w->rows, K = w->cols;
+  if (M < 1 || N % 8 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
+      (T_save && !aligned16(T_save)))
+    return QLORA_ERR_ALIGN;
+  const FwdWs lay = fwd_ws(M, N, r);
+  if (!ws || ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  st = current_device(&d);
+  if (st) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int RP = padded_rank(r);
+  const float scale = alpha / (float)r;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  void* sT = wsb + lay.sT;
+  const void* Bp = B;
+  if (r < RP) {
+    launch_pad_cols(B, (int)N, r, RP, wsb + lay.Bpad, s);
+    Bp = wsb + lay.Bpad;
+  }
+  launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save, s);
+  FwdArgs a{};
+  a.packed = w->packed;
+  a.absmax = w->absmax;
+  a.qabsmax = w->qabsmax;
+  a.dq_scale = w->dq_scale;
+  a.dq_mean = w->dq_mean;
+  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.M = (int)M; a.N = (int)N; a.K = (int)K;
+  a.na = RP / 64;
+  a.double_quant = w->double_quant;
+  a.status = d->status;
+  for (int i = 0; i < 16; ++i) a.q[i] = host_tables().q[i];
+  st = launch_qlora_fwd_gemm(a, X, sT, Bp, RP, s, d->sms);
+  if (st) return st;
+  return launch_status();
 }
 
 int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,

@@ -1,0 +1,132 @@
+"""GPU parity of the QLoRA linear layer (forward, backward) against the oracle.
+
+Bar: max|GPU - oracle| / max|oracle| <= 1e-2 per output tensor (bf16 inputs,
+fp32 accumulation, bf16 outputs; the oracle is fp64 on the same bf16 inputs
+and the oracle's own dequantised weight, which the quantisation tests show
+equals the GPU's bit for bit).  The bf16 rounding of the output alone is
+2^-9 relative; a dropped adapter term is >= 4 % of max|Y| on these
+workloads, so the bar separates right from wrong.
+
+Two cases are exact: with X = identity and A = 0 the forward returns the
+in-GEMM dequantised weights, which must equal nf4_dequantize bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qlora_linear_layers_b200 import synth
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def q():
+    from qlora_linear_layers_b200.build import build
+    build()
+    import qlora_linear_layers_b200 as q
+    return q
+
+
+def rel_err(got, ref):
+    g = got.float().cpu().numpy().astype(np.float64) if torch.is_tensor(got) else got
+    return float(np.max(np.abs(g - ref)) / np.max(np.abs(ref)))
+
+
+def _oracle_weight(wq, W_cpu):
+    codes, a = oracle.quantize(W_cpu.float().numpy())
+    if wq.double_quant:
+        qa, s, mu = oracle.double_quantize(a)
+        a = oracle.dq_absmax(qa, s, mu)
+    return oracle.dequantize(oracle.pack(codes), a, tuple(W_cpu.shape))
+
+
+def _layer(q, N, K, M, r, alpha, seed, dq=True, wdtype="bf16"):
+    W = synth.weight(N, K, seed + 1, wdtype)
+    X = synth.activations(M, K, seed + 2)
+    A = synth.activations(r, K, seed + 3, sigma=0.02)
+    B = synth.activations(N, r, seed + 4, sigma=0.02)
+    wq = q.quantize(W.cuda(), double_quant=dq)
+    return W, X, A, B, wq
+
+
+@pytest.mark.parametrize("N,K,M,r,alpha,dq", [
+    (1024, 1024, 16, 8, 16.0, True),       # tiny round-trip workload
+    (1024, 1024, 16, 8, 16.0, False),
+    (200, 192, 300, 16, 32.0, True),       # ragged N and M tiles, 3 K steps
+    (384, 512, 257, 32, 8.0, True),
+    (256, 640, 513, 64, 16.0, True),
+    (136, 256, 700, 128, 64.0, False),
+    (512, 1024, 1, 16, 32.0, True),        # decode-sized token counts
+    (512, 1024, 4, 16, 32.0, True),
+    (512, 1024, 17, 16, 32.0, True),
+])
+def test_forward_small(q, N, K, M, r, alpha, dq):
+    W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=100 * M + r, dq=dq, wdtype="bf16")
+    Y, T = q.linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), alpha)
+    assert q.qlora_check_status() == 0
+    Wd = _oracle_weight(wq, W)
+    Yr, Tr = oracle.linear_fwd(X.float().numpy(), Wd, A.float().numpy(), B.float().numpy(), alpha, r)
+    assert rel_err(Y, Yr) <= TOL
+    assert rel_err(T, Tr) <= TOL
+
+
+def test_forward_identity_is_exact_dequant(q):
+    """X = I, A = 0: Y[m, n] = W'[n, m] exactly (one nonzero product per sum)."""
+    N, K = 384, 512
+    W = synth.weight(N, K, 4242, "bf16")
+    wq = q.quantize(W.cuda(), double_quant=True)
+    X = torch.eye(K, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
+    B = synth.activations(N, 16, 4243, sigma=0.02).cuda()
+    Y, _ = q.linear_fwd(wq, X, A, B, 32.0)
+    Wdeq = q.dequantize(wq)
+    assert q.qlora_check_status() == 0
+    assert torch.equal(Y.t().contiguous().view(torch.int16), Wdeq.view(torch.int16))
+    Wd = _oracle_weight(wq, W)
+    assert np.array_equal(Y.t().float().cpu().numpy(), Wd)
+
+
+def test_forward_adapter_only(q):
+    """W = 0 quantises to the exact-zero row everywhere: Y = s (X A^T) B^T."""
+    N, K, M, r, alpha = 256, 512, 300, 16, 32.0
+    W = torch.zeros(N, K, dtype=torch.bfloat16)
+    X = synth.activations(M, K, 5001)
+    A = synth.activations(r, K, 5002, sigma=0.02)
+    B = synth.activations(N, r, 5003, sigma=0.02)
+    wq = q.quantize(W.cuda(), double_quant=True)
+    Y, _ = q.linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), alpha)
+    assert q.qlora_check_status() == 0
+    Yr, _ = oracle.linear_fwd(X.float().numpy(), np.zeros((N, K)), A.float().numpy(),
+                              B.float().numpy(), alpha, r)
+    assert rel_err(Y, Yr) <= TOL
+
+
+def _sampled_forward(q, W, X, A, B, alpha, r, nrows=48, seed=0):
+    wq = q.quantize(W.cuda(), double_quant=True)
+    Y, T = q.linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), alpha)
+    assert q.qlora_check_status() == 0
+    rng = np.random.default_rng(seed)
+    M = X.shape[0]
+    rows = np.unique(np.concatenate([rng.choice(M, nrows, replace=False), [0, M - 1]]))
+    Wd = _oracle_weight(wq, W)
+    Yr, _ = oracle.linear_fwd(X[rows].float().numpy(), Wd, A.float().numpy(), B.float().numpy(),
+                              alpha, r)
+    assert rel_err(Y[rows], Yr) <= TOL
+
+
+@pytest.mark.slow
+def test_forward_attn_proj_full_size_sampled(q):
+    wl = synth.WORKLOADS["attn_proj_4096"]
+    W, X, A, B = synth.layer_inputs(wl, 0)
+    _sampled_forward(q, W, X, A, B, wl.alpha, wl.r)
+
+
+@pytest.mark.slow
+def test_forward_mlp_7b_full_size_sampled(q):
+    wl = synth.WORKLOADS["mlp_7b"]
+    for which in range(3):
+        W, X, A, B = synth.layer_inputs(wl, which)
+        _sampled_forward(q, W, X, A, B, wl.alpha, wl.r, seed=which)
