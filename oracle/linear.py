@@ -53,3 +53,17 @@ def linear_bwd(X, dY, Wdeq, A, B, alpha: float, r: int):
     dA = s * (U.T @ X)
     dB = s * (dY.T @ (X @ A.T))
     return dX, dA, dB
+
+
+def linear_bwd_adapters(X, dY, A, B, alpha: float, r: int):
+    """dA = s (dY B)^T X and dB = s dY^T (X A^T) alone (no dX), fp64.
+
+    Same formulas as linear_bwd; split out so that the adapter gradients of a
+    large layer can be checked in full without forming the M x N x K product
+    that dX needs.
+    """
+    X, dY, A, B = _f64(X), _f64(dY), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    dA = s * ((dY @ B).T @ X)
+    dB = s * (dY.T @ (X @ A.T))
+    return dA, dB

@@ -76,6 +76,26 @@ FwdWs fwd_ws(int64_t M, int64_t N, int r) {
   return w;
 }
 
+// Backward workspace, in order: T [M, r] (recomputed when not passed),
+// sU [M, RP], Wt = deq(W)^T [K, N], At = A^T [K, RP] (all bf16), then the
+// fp32 split-M partial sums of dA and dB.
+struct BwdWs {
+  size_t T, sU, Wt, At, pA, pB, total;
+};
+BwdWs bwd_ws(int64_t M, int64_t N, int64_t K, int r) {
+  BwdWs w{};
+  const int RP = padded_rank(r);
+  size_t off = 0;
+  w.T = off;  off += align256((size_t)M * r * 2);
+  w.sU = off; off += align256((size_t)M * RP * 2);
+  w.Wt = off; off += align256((size_t)K * N * 2);
+  w.At = off; off += align256((size_t)K * RP * 2);
+  w.pA = off; off += align256(atb_workspace_floats(r, (int)K, (int)M) * 4);
+  w.pB = off; off += align256(atb_workspace_floats((int)N, r, (int)M) * 4);
+  w.total = off;
+  return w;
+}
+
 int launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
@@ -147,6 +167,9 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     case QLORA_OP_FWD:
       if (M < 1 || N < 1 || !valid_rank(r)) return 0;
       return fwd_ws(M, N, r).total;
+    case QLORA_OP_BWD:
+      if (M < 1 || N < 1 || K < 1 || !valid_rank(r)) return 0;
+      return bwd_ws(M, N, K, r).total;
     default: return 0;
   }
 }
@@ -226,19 +249,19 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
     Bp = wsb + lay.Bpad;
   }
   launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save, s);
-  FwdArgs a{};
+  GemmArgs a{};
   a.packed = w->packed;
   a.absmax = w->absmax;
   a.qabsmax = w->qabsmax;
   a.dq_scale = w->dq_scale;
   a.dq_mean = w->dq_mean;
-  a.Y = static_cast<__nv_bfloat16*>(Y);
-  a.M = (int)M; a.N = (int)N; a.K = (int)K;
+  a.out = static_cast<__nv_bfloat16*>(Y);
+  a.Mtok = (int)M; a.Nout = (int)N; a.Kc = (int)K;
   a.na = RP / 64;
   a.double_quant = w->double_quant;
   a.status = d->status;
   for (int i = 0; i < 16; ++i) a.q[i] = host_tables().q[i];
-  st = launch_qlora_fwd_gemm(a, X, sT, Bp, RP, s, d->sms);
+  st = launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
   if (st) return st;
   return launch_status();
 }
@@ -246,9 +269,50 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
 int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
                      const void* B, int r, float alpha, const void* T, void* dX, void* dA,
                      void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  (void)w; (void)X; (void)dY; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)T;
-  (void)dX; (void)dA; (void)dB; (void)ws; (void)ws_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  int st = check_weight(w);
+  if (st) return st;
+  if (!X || !dY || !A || !B || !dX || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!valid_rank(r) || !(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return QLORA_ERR_INVALID_ARG;
+  const int64_t N = w->rows, K = w->cols;
+  if (M < 1 || N % 8 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(A) || !aligned16(B) || !aligned16(dX) ||
+      !aligned16(dA) || !aligned16(dB) || (T && !aligned16(T)))
+    return QLORA_ERR_ALIGN;
+  const BwdWs lay = bwd_ws(M, N, K, r);
+  if (!ws || ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  st = current_device(&d);
+  if (st) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int RP = padded_rank(r);
+  const float scale = alpha / (float)r;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  void* Tw = wsb + lay.T;
+  void* sU = wsb + lay.sU;
+  void* Wt = wsb + lay.Wt;
+  void* At = wsb + lay.At;
+  if (!T) {
+    launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, nullptr, Tw, s);
+    T = Tw;
+  }
+  launch_lora_u(dY, B, (int)M, (int)N, r, RP, scale, sU, s);
+  launch_dequant_t(w, Wt, s);
+  launch_transpose_pad(A, r, (int)K, RP, At, s);
+  // dX[M, K] = dY Wt^T + sU At^T   (tokens = dY rows, outputs = K, contraction = N)
+  GemmArgs a{};
+  a.out = static_cast<__nv_bfloat16*>(dX);
+  a.Mtok = (int)M; a.Nout = (int)K; a.Kc = (int)N;
+  a.na = RP / 64;
+  a.status = d->status;
+  st = launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
+  if (st) return st;
+  // dA[r, K] = (s U)^T X ;  dB[N, r] = s dY^T T
+  launch_atb(sU, RP, r, X, (int)K, (int)K, (int)M, 1.0f, dA, reinterpret_cast<float*>(wsb + lay.pA),
+             d->sms, s);
+  launch_atb(dY, (int)N, (int)N, T, r, r, (int)M, scale, dB, reinterpret_cast<float*>(wsb + lay.pB),
+             d->sms, s);
+  return launch_status();
 }
 
 int qlora_check_status(qlora_stream_t stream) {

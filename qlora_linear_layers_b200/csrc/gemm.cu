@@ -1,0 +1,409 @@
+// Tensor-core GEMM engine of the QLoRA layer (tcgen05 / TMEM / TMA, sm_100a).
+//
+//   out[m, o] = sum_c tok[m, c] * Wt[o, c]  +  sum_j tokad[m, j] * Wad[o, j]
+//
+// computed transposed (out^T = Wt tok^T) so that the weight side is the MMA's
+// A operand (128 rows per tile) and the token side its B operand (256 tokens
+// per tile).  Two modes:
+//
+//  MODE_NF4 (forward, Y = X deq(W)^T + (s T) B^T).  Page "QLoRA Explained",
+//    section "Why the expansion cannot be skipped": the tensor core cannot
+//    decode a 4-bit row index, so a kernel reads the codes, looks them up in
+//    the 16-entry table, multiplies by the block scale and hands bf16 to the
+//    tensor core.  Here converter warps do that for one weight row per thread
+//    and one NF4 block per K step (64 = the block size): a 16-entry bf16 table
+//    per block is built in registers as two byte planes, codes are expanded
+//    with prmt, and the bf16 row goes straight into a tensor-memory ring with
+//    tcgen05.st -- tcgen05.mma reads A from TMEM, so the dequantised weights
+//    never touch shared memory.
+//
+//  MODE_BF16 (backward dX = dY deq(W) + (s U) A).  Both operands arrive by
+//    TMA; the weight side is deq(W)^T prepared by a dequantise-transpose pass.
+//
+// The adapter term (page "LoRA vs QLoRA", section "How LoRA Works": W' = W +
+// (alpha/r) B A) is ceil(r/64) extra K steps of an SS MMA into the same TMEM
+// accumulator, with the rank padded to 64 by zeros.
+//
+// Persistent: one CTA per SM walks a static tile schedule.  Warp 0 issues
+// TMA, warp 1 issues MMA, warps 2-9 drain the accumulator (two warps per TMEM
+// lane quadrant, 128 columns each), warps 10-13 convert NF4 (MODE_NF4).  The
+// accumulator is released as soon as it sits in registers, so the next tile's
+// MMAs overlap the stores.  Every wait is bounded (status QLORA_ERR_TIMEOUT).
+
+#include <algorithm>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "gemm.h"
+
+namespace qnf4 {
+
+namespace eng {
+
+constexpr int BN = 128;          // weight-side rows per tile (MMA M)
+constexpr int BM = 256;          // tokens per tile (MMA N)
+constexpr int BK = 64;           // contraction per stage (= one NF4 block)
+constexpr int STAGES = 4;
+constexpr int MAX_NA = 2;        // adapter K steps (r <= 128)
+constexpr int X_BYTES = BM * BK * 2;            // 32 KB token tile
+constexpr int W_BYTES = BN * BK * 2;            // 16 KB weight tile
+constexpr int ACC_COL = 0;                      // accumulator: TMEM columns [0, 256)
+constexpr int A_COL = 256;                      // NF4 A ring: STAGES x 32 columns
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 448;                // 14 warps
+constexpr int EPI_WARP0 = 2;
+constexpr int CVT_WARP0 = 10;
+
+template <int MODE>
+struct Smem {
+  uint8_t x[STAGES][X_BYTES];
+  // MODE_NF4: adapter weight tiles;  MODE_BF16: weight tile of each stage
+  uint8_t w[MODE == MODE_NF4 ? MAX_NA : STAGES][W_BYTES];
+  uint64_t x_full[STAGES], x_empty[STAGES];
+  uint64_t a_full[STAGES], a_empty[STAGES];
+  uint64_t aux_full[MAX_NA], aux_empty[MAX_NA];
+  uint64_t acc_full, acc_empty, done;
+  uint32_t tmem_base;
+  int abort;
+  float inv127[256];
+};
+
+template <int MODE>
+constexpr size_t smem_bytes() { return sizeof(Smem<MODE>) + 1024; }
+
+// 16-entry bf16 table for one block, held as byte planes: L[i] holds the low
+// bytes of entries 4i..4i+3, H[i] the high bytes.
+struct Lut { uint32_t L[4], H[4]; };
+
+__device__ __forceinline__ Lut build_lut(float a, const float* q) {
+  uint32_t P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    P[i] = pack_bf16x2(__fmul_rn(q[2 * i], a), __fmul_rn(q[2 * i + 1], a));
+  Lut l;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    l.L[i] = prmt(P[2 * i], P[2 * i + 1], 0x6420);
+    l.H[i] = prmt(P[2 * i], P[2 * i + 1], 0x7531);
+  }
+  return l;
+}
+
+// Expand one 32-bit word of packed codes (8 weights, byte j = element 2j in
+// the high nibble, 2j+1 in the low nibble) into 4 bf16x2 words ordered by K.
+__device__ __forceinline__ void lookup8(uint32_t w, const Lut& l, uint32_t* out) {
+  const uint32_t s7 = w & 0x77777777u;                       // entry index within a plane half
+  const uint32_t t = ((w >> 1) & 0x44444444u) | 0x32103210u; // pick half 0-7 or 8-15 per byte
+  {
+    const uint32_t xl = prmt(l.L[0], l.L[1], s7), yl = prmt(l.L[2], l.L[3], s7);
+    const uint32_t xh = prmt(l.H[0], l.H[1], s7), yh = prmt(l.H[2], l.H[3], s7);
+    const uint32_t lo = prmt(xl, yl, t), hi = prmt(xh, yh, t);
+    out[0] = prmt(lo, hi, 0x4051);
+    out[1] = prmt(lo, hi, 0x6273);
+  }
+  {
+    const uint32_t s7h = s7 >> 16, th = t >> 16;
+    const uint32_t xl = prmt(l.L[0], l.L[1], s7h), yl = prmt(l.L[2], l.L[3], s7h);
+    const uint32_t xh = prmt(l.H[0], l.H[1], s7h), yh = prmt(l.H[2], l.H[3], s7h);
+    const uint32_t lo = prmt(xl, yl, th), hi = prmt(xh, yh, th);
+    out[2] = prmt(lo, hi, 0x4051);
+    out[3] = prmt(lo, hi, 0x6273);
+  }
+}
+
+template <int MODE, bool DQ>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
+             const __grid_constant__ CUtensorMap tm_tokad,   // [Mtok, RP]  bf16
+             const __grid_constant__ CUtensorMap tm_wad,     // [Nout, RP]  bf16
+             const __grid_constant__ CUtensorMap tm_w,       // [Nout, Kc]  bf16 (MODE_BF16)
+             const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<MODE>& S =
+      *reinterpret_cast<Smem<MODE>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int n_tiles_n = (p.Nout + BN - 1) / BN;
+  const int n_tiles = n_tiles_n * ((p.Mtok + BM - 1) / BM);
+  const int nk = (p.Kc + BK - 1) / BK;
+  const int na = p.na;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&S.x_full[i], 1);
+      mbar_init(&S.x_empty[i], 1);
+      mbar_init(&S.a_full[i], 128);
+      mbar_init(&S.a_empty[i], 1);
+    }
+    for (int i = 0; i < MAX_NA; ++i) { mbar_init(&S.aux_full[i], 1); mbar_init(&S.aux_empty[i], 1); }
+    mbar_init(&S.acc_full, 1);
+    mbar_init(&S.acc_empty, 256);
+    mbar_init(&S.done, 1);
+    S.abort = 0;
+    mbar_fence_init();
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    S.inv127[i] = __fdiv_rn((float)(i - 127), 127.0f);
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_tok);
+    tma_prefetch_desc(&tm_tokad);
+    tma_prefetch_desc(&tm_wad);
+    if (MODE == MODE_BF16) tma_prefetch_desc(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t xi = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+        const int n0 = (tile % n_tiles_n) * BN;
+        const int m0 = (tile / n_tiles_n) * BM;
+        for (int ks = 0; ks < nk + na; ++ks, ++xi) {
+          const int s = xi % STAGES;
+          if (!(ok = mbar_wait(&S.x_empty[s], ((xi / STAGES) & 1) ^ 1, abort, p.status))) break;
+          if (MODE == MODE_BF16) {
+            mbar_arrive_expect_tx(&S.x_full[s], X_BYTES + W_BYTES);
+            if (ks < nk) {
+              tma_load_2d(S.x[s], &tm_tok, &S.x_full[s], ks * BK, m0);
+              tma_load_2d(S.w[s], &tm_w, &S.x_full[s], ks * BK, n0);
+            } else {
+              tma_load_2d(S.x[s], &tm_tokad, &S.x_full[s], (ks - nk) * BK, m0);
+              tma_load_2d(S.w[s], &tm_wad, &S.x_full[s], (ks - nk) * BK, n0);
+            }
+          } else {
+            mbar_arrive_expect_tx(&S.x_full[s], X_BYTES);
+            if (ks < nk) {
+              tma_load_2d(S.x[s], &tm_tok, &S.x_full[s], ks * BK, m0);
+            } else {
+              const int j = ks - nk;
+              tma_load_2d(S.x[s], &tm_tokad, &S.x_full[s], j * BK, m0);
+              if (!(ok = mbar_wait(&S.aux_empty[j], (lt & 1) ^ 1, abort, p.status))) break;
+              mbar_arrive_expect_tx(&S.aux_full[j], W_BYTES);
+              tma_load_2d(S.w[j], &tm_wad, &S.aux_full[j], j * BK, n0);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BN, BM);
+      uint32_t xi = 0, ai = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+        ok = mbar_wait(&S.acc_empty, (lt & 1) ^ 1, abort, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nk && ok; ++ks, ++xi) {
+          const int s = xi % STAGES;
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
+          if (MODE == MODE_NF4) {
+            const int sa = ai % STAGES;
+            ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status) &&
+                 mbar_wait(&S.a_full[sa], (ai / STAGES) & 1, abort, p.status);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_ts(tmem + ACC_COL, tmem + A_COL + sa * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
+                     idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&S.x_empty[s]);
+            mma_commit(&S.a_empty[sa]);
+            ++ai;
+          } else {
+            ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[s]));
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_ss(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
+                     (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&S.x_empty[s]);
+          }
+        }
+        for (int j = 0; j < na && ok; ++j, ++xi) {
+          const int s = xi % STAGES;
+          ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status);
+          if (ok && MODE == MODE_NF4) ok = mbar_wait(&S.aux_full[j], lt & 1, abort, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[MODE == MODE_NF4 ? j : s]));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ss(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, 1u);
+          mma_commit(&S.x_empty[s]);
+          if (MODE == MODE_NF4) mma_commit(&S.aux_empty[j]);
+        }
+        if (ok) mma_commit(&S.acc_full);
+      }
+      // all MMAs issued by this thread are complete once `done` flips
+      mma_commit(&S.done);
+      mbar_wait(&S.done, 0, abort, p.status);
+    }
+  } else if (warp >= CVT_WARP0) {
+    // ------------------------------------------------------------ NF4 -> bf16 converters
+    if (MODE == MODE_NF4) {
+      const int quad = warp & 3;
+      const int row_in_tile = quad * 32 + lane;
+      const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
+      const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
+      const int64_t kb_per_row = p.Kc / 64;
+      uint32_t ai = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int n = (tile % n_tiles_n) * BN + row_in_tile;
+        const bool valid = n < p.Nout;
+        const uint4* codes =
+            reinterpret_cast<const uint4*>(p.packed + (int64_t)(valid ? n : 0) * (p.Kc / 2));
+        const int64_t blk0 = (int64_t)(valid ? n : 0) * kb_per_row;
+        // software pipeline: data for step ks+1 is loaded while step ks converts
+        uint4 c0 = __ldcg(codes), c1 = __ldcg(codes + 1);
+        float a_raw = 0.0f;
+        int qa = 0;
+        if (DQ) qa = __ldcg(p.qabsmax + blk0); else a_raw = __ldcg(p.absmax + blk0);
+        float sg = DQ ? __ldg(p.dq_scale + (blk0 >> 8)) : 0.0f;
+        for (int ks = 0; ks < nk; ++ks, ++ai) {
+          uint4 n0v = c0, n1v = c1;
+          int nqa = qa;
+          float na_raw = a_raw, nsg = sg;
+          if (ks + 1 < nk) {
+            n0v = __ldcg(codes + 2 * (ks + 1));
+            n1v = __ldcg(codes + 2 * (ks + 1) + 1);
+            const int64_t b = blk0 + ks + 1;
+            if (DQ) { nqa = __ldcg(p.qabsmax + b); nsg = __ldg(p.dq_scale + (b >> 8)); }
+            else na_raw = __ldcg(p.absmax + b);
+          }
+          // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
+          const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[qa + 127], sg), mu) : a_raw;
+          uint32_t v[32];
+          if (valid) {
+            const Lut l = build_lut(a, p.q);
+            const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          const int sa = ai % STAGES;
+          if (!mbar_wait(&S.a_empty[sa], ((ai / STAGES) & 1) ^ 1, abort, p.status)) { ok = false; break; }
+          __syncwarp();
+          tc_fence_after();
+          const uint32_t taddr = tmem + tmem_lane + A_COL + sa * 32;
+          tmem_st16(taddr, v);
+          tmem_st16(taddr + 16, v + 16);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&S.a_full[sa]);
+          c0 = n0v; c1 = n1v; qa = nqa; a_raw = na_raw; sg = nsg;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    constexpr int COLS = BM / 2;                 // accumulator columns per epilogue warp
+    const int quad = warp & 3;
+    const int col0 = ((warp - EPI_WARP0) >> 2) * COLS;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
+    uint32_t lt = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
+      const int n0 = (tile % n_tiles_n) * BN;
+      const int m0 = (tile / n_tiles_n) * BM + col0;
+      if (!mbar_wait(&S.acc_full, lt & 1, abort, p.status)) break;
+      __syncwarp();
+      tc_fence_after();
+      uint32_t packed[COLS / 2];
+#pragma unroll
+      for (int c = 0; c < COLS; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + tmem_lane + ACC_COL + col0 + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          packed[c / 2 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+      }
+      tc_fence_before();
+      mbar_arrive(&S.acc_empty);
+      // lane pairs (o, o+1) swap halves so each lane stores two adjacent
+      // outputs of one token row: even lanes row m, odd lanes row m+1
+      const bool odd = lane & 1;
+      const int ocol = n0 + row_in_tile - (odd ? 1 : 0);
+      const int mfirst = m0 + (odd ? 1 : 0);
+      const int rows_left = (ocol < p.Nout) ? p.Mtok - mfirst : 0;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (int64_t)mfirst * p.Nout + ocol);
+      const int step = p.Nout;                   // two bf16 rows = Nout words
+#pragma unroll
+      for (int c = 0; c < COLS; c += 2) {
+        const uint32_t mine = packed[c / 2];
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+        const uint32_t out = odd ? prmt(other, mine, 0x7632) : prmt(mine, other, 0x5410);
+        if (c < rows_left) *dst = out;
+        dst += step;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int MODE, bool DQ>
+static void launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                       const CUtensorMap& d, const GemmArgs& p, int grid, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_qlora_gemm<MODE, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<MODE>());
+    attr = true;
+  }
+  k_qlora_gemm<MODE, DQ><<<grid, NUM_THREADS, smem_bytes<MODE>(), s>>>(a, b, c, d, p);
+}
+
+}  // namespace eng
+
+int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* tokad,
+                      const void* wad, const void* w, int RP, cudaStream_t s, int num_sms) {
+  using namespace eng;
+  CUtensorMap t_tok, t_tokad, t_wad, t_w;
+  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, BM)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, BM)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_wad, wad, RP, a.Nout, RP, BK, BN)) return QLORA_ERR_CUDA;
+  if (mode == MODE_BF16) {
+    if (!make_tmap_2d_bf16(&t_w, w, a.Kc, a.Nout, a.Kc, BK, BN)) return QLORA_ERR_CUDA;
+  } else {
+    t_w = t_wad;                                  // unused
+  }
+  const int n_tiles = ((a.Nout + BN - 1) / BN) * ((a.Mtok + BM - 1) / BM);
+  const int grid = std::min(n_tiles, num_sms);
+  if (mode == MODE_BF16)
+    launch_one<MODE_BF16, false>(t_tok, t_tokad, t_wad, t_w, a, grid, s);
+  else if (a.double_quant)
+    launch_one<MODE_NF4, true>(t_tok, t_tokad, t_wad, t_w, a, grid, s);
+  else
+    launch_one<MODE_NF4, false>(t_tok, t_tokad, t_wad, t_w, a, grid, s);
+  return cudaGetLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace qnf4

@@ -6,25 +6,32 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "../../include/qlora_nf4.h"
+
 namespace qnf4 {
 
-// Fused NF4 forward GEMM: Y[M, N] = X deq(W)^T + (s T) B^T.
-struct FwdArgs {
-  const uint8_t* packed;      // [N, K/2]
-  const float* absmax;        // [N*K/64]       (double_quant == 0)
-  const int8_t* qabsmax;      // [N*K/64]       (double_quant == 1)
-  const float* dq_scale;      // [ceil(N*K/64/256)]
+constexpr int MODE_NF4 = 0;    // weight side dequantised from NF4 into TMEM
+constexpr int MODE_BF16 = 1;   // weight side is a bf16 matrix loaded by TMA
+
+// out[Mtok, Nout] = tok[Mtok, Kc] Wt[Nout, Kc]^T + tokad[Mtok, RP] Wad[Nout, RP]^T
+struct GemmArgs {
+  // MODE_NF4 weight (Wt = deq(W), W is [Nout, Kc])
+  const uint8_t* packed;      // [Nout, Kc/2]
+  const float* absmax;        // [Nout*Kc/64]     (double_quant == 0)
+  const int8_t* qabsmax;      // [Nout*Kc/64]     (double_quant == 1)
+  const float* dq_scale;      // [ceil(Nout*Kc/64/256)]
   const float* dq_mean;       // [1]
-  __nv_bfloat16* Y;           // [M, N]
-  int M, N, K;
-  int na;                     // adapter K steps = ceil(r / 64)
+  __nv_bfloat16* out;         // [Mtok, Nout]
+  int Mtok, Nout, Kc;
+  int na;                     // adapter K steps = RP / 64
   int double_quant;
   int* status;
   float q[16];                // NF4 table
 };
 
-int launch_qlora_fwd_gemm(const FwdArgs& a, const void* X, const void* sT, const void* Bpad,
-                          int RP, cudaStream_t s, int num_sms);
+// tok: [Mtok, Kc]; tokad: [Mtok, RP]; wad: [Nout, RP]; w: [Nout, Kc] (MODE_BF16 only).
+int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* tokad,
+                      const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);
 
 // 2-D bf16 tensor map, 128-byte swizzle, box [box_outer rows x box_inner cols].
 bool make_tmap_2d_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
@@ -35,6 +42,22 @@ bool make_tmap_2d_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64
 //   T_save[M, r]  = RNbf16(T)      (if not null)
 void launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
                       void* sT_pad, void* T_save, cudaStream_t st);
+
+// U = dY B:  sU_pad[M, RP] = RNbf16(s * U), zero beyond r.
+void launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
+                   void* sU_pad, cudaStream_t st);
+
+// C[Rdim, Cdim] = RNbf16(s * P^T Q) over M token rows, split over the tokens
+// into fixed chunks summed in order; `part` holds atb_workspace_floats floats.
+void launch_atb(const void* P, int ldp, int Rdim, const void* Q, int ldq, int Cdim, int M, float s,
+                void* out, float* part, int num_sms, cudaStream_t st);
+size_t atb_workspace_floats(int Rdim, int Cdim, int M);
+
+// Wt[K, N] = deq(W)^T (bf16, the values of nf4_dequantize).
+void launch_dequant_t(const nf4_weight* w, void* Wt, cudaStream_t st);
+
+// At[K, RP] = A[r, K]^T zero-padded to RP columns.
+void launch_transpose_pad(const void* A, int r, int K, int RP, void* At, cudaStream_t st);
 
 // Bpad[N, RP] = B[N, r] zero-padded to RP columns.
 void launch_pad_cols(const void* B, int rows, int r, int RP, void* Bpad, cudaStream_t st);

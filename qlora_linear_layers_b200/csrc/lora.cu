@@ -48,33 +48,57 @@ __device__ __forceinline__ uint32_t swz64(int row, int k) {
   return (uint32_t)(row * 128 + ((((k >> 3) ^ (row & 7))) << 4) + ((k & 7) << 1));
 }
 
+// Byte offset of element (row, col) in a [rows][W] bf16 tile (W = 64 or 128)
+// whose 16-byte chunks are XOR-swizzled by row.
+template <int W>
+__device__ __forceinline__ uint32_t swzw(int row, int col) {
+  return (uint32_t)(row * W * 2 + ((((col >> 3) ^ (row & 7))) << 4) + ((col & 7) << 1));
+}
+
 // ===========================================================================
-// T = X A^T : CTA = 64 tokens x RP adapter columns, 4 warps x 16 tokens.
+// Skinny product  S[M, RP] = Z[M, L] * R   (R = A^T or B; rank <= 128)
+//   BT = false: R[l, j] = A[j, l]   (A is [r, L], L contiguous)   -> T = X A^T
+//   BT = true : R[l, j] = B[l, j]   (B is [L, r], r contiguous)   -> U = dY B
+// CTA = 64 rows of Z x RP columns, 4 warps x 16 rows, L in chunks of 64.
+// Outputs: Ss[M, RP] = RNbf16(s * S) (zero beyond r), Sraw[M, r] = RNbf16(S).
 // ===========================================================================
-template <int RP>
+template <int RP, bool BT>
 __global__ void __launch_bounds__(128)
-k_lora_down(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M,
-            int K, int r, float s, __nv_bfloat16* __restrict__ sT, __nv_bfloat16* __restrict__ Tsave) {
+k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restrict__ R, int M,
+              int L, int r, float s, __nv_bfloat16* __restrict__ Ss, __nv_bfloat16* __restrict__ Sraw) {
   constexpr int TM = 64, KC = 64, STG = 3;
   constexpr int XB = TM * KC * 2, AB = RP * KC * 2;
   extern __shared__ __align__(128) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * TM;
-  const int nkc = K / KC;
+  const int nkc = (L + KC - 1) / KC;
 
   auto load_stage = [&](int kc, int stg) {
     uint8_t* xs = sm + stg * (XB + AB);
     uint8_t* as = xs + XB;
     for (int c = tid; c < TM * 8; c += 128) {
       const int row = c >> 3, ch = c & 7;
-      const int m = m0 + row;
-      const __nv_bfloat16* g = X + (int64_t)(m < M ? m : 0) * K + kc * KC + ch * 8;
-      cp_async16(smem_u32(xs) + swz64(row, ch * 8), g, m < M ? 16 : 0);
+      const int m = m0 + row, l = kc * KC + ch * 8;
+      const bool ok = m < M && l < L;
+      cp_async16(smem_u32(xs) + swz64(row, ch * 8), ok ? (const void*)(Z + (int64_t)m * L + l) : (const void*)Z,
+                 ok ? 16 : 0);
     }
-    for (int c = tid; c < RP * 8; c += 128) {
-      const int row = c >> 3, ch = c & 7;
-      const __nv_bfloat16* g = A + (int64_t)(row < r ? row : 0) * K + kc * KC + ch * 8;
-      cp_async16(smem_u32(as) + swz64(row, ch * 8), g, row < r ? 16 : 0);
+    if (!BT) {
+      for (int c = tid; c < RP * 8; c += 128) {
+        const int row = c >> 3, ch = c & 7;            // row = j, chunk along l
+        const int l = kc * KC + ch * 8;
+        const bool ok = row < r && l < L;
+        cp_async16(smem_u32(as) + swz64(row, ch * 8), ok ? (const void*)(R + (int64_t)row * L + l) : (const void*)R,
+                   ok ? 16 : 0);
+      }
+    } else {
+      for (int c = tid; c < KC * (RP / 8); c += 128) {
+        const int row = c / (RP / 8), ch = c % (RP / 8);   // row = l, chunk along j
+        const int l = kc * KC + row;
+        const bool ok = l < L && ch * 8 < r;
+        cp_async16(smem_u32(as) + swzw<RP>(row, ch * 8), ok ? (const void*)(R + (int64_t)l * r + ch * 8) : (const void*)R,
+                   ok ? 16 : 0);
+      }
     }
   };
 
@@ -105,9 +129,15 @@ k_lora_down(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict
 #pragma unroll
       for (int pr = 0; pr < RP / 16; ++pr) {
         uint32_t b0, b1, b2, b3;
-        const int row = pr * 16 + (lane & 7) + 8 * (lane >> 4);
-        const int k = k16 * 16 + 8 * ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(as) + swz64(row, k), b0, b1, b2, b3);
+        if (!BT) {
+          const int row = pr * 16 + (lane & 7) + 8 * (lane >> 4);
+          const int k = k16 * 16 + 8 * ((lane >> 3) & 1);
+          ldsm_x4(smem_u32(as) + swz64(row, k), b0, b1, b2, b3);
+        } else {
+          const int row = k16 * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+          const int col = pr * 16 + 8 * (lane >> 4);
+          ldsm_x4_t(smem_u32(as) + swzw<RP>(row, col), b0, b1, b2, b3);
+        }
         mma_bf16_16816(acc[2 * pr], a0, a1, a2, a3, b0, b1);
         mma_bf16_16816(acc[2 * pr + 1], a0, a1, a2, a3, b2, b3);
       }
@@ -124,31 +154,290 @@ k_lora_down(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict
       const int m = m0 + warp * 16 + g + 8 * h;
       if (m >= M) continue;
       const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
-      *reinterpret_cast<uint32_t*>(sT + (int64_t)m * RP + col) =
-          pack_bf16x2(__fmul_rn(s, v0), __fmul_rn(s, v1));
-      if (Tsave && col < r)
-        *reinterpret_cast<uint32_t*>(Tsave + (int64_t)m * r + col) = pack_bf16x2(v0, v1);
+      if (Ss)
+        *reinterpret_cast<uint32_t*>(Ss + (int64_t)m * RP + col) =
+            pack_bf16x2(__fmul_rn(s, v0), __fmul_rn(s, v1));
+      if (Sraw && col < r)
+        *reinterpret_cast<uint32_t*>(Sraw + (int64_t)m * r + col) = pack_bf16x2(v0, v1);
     }
   }
 }
 
+template <int RP, bool BT>
+static void launch_skinny(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
+                          void* Sraw, cudaStream_t st) {
+  constexpr int smem = 3 * (64 * 64 * 2 + RP * 64 * 2);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_lora_skinny<RP, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr = true;
+  }
+  k_lora_skinny<RP, BT><<<(M + 63) / 64, 128, smem, st>>>(
+      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)R, M, L, r, s, (__nv_bfloat16*)Ss,
+      (__nv_bfloat16*)Sraw);
+}
+
 void launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
                       void* sT_pad, void* T_save, cudaStream_t st) {
-  const int grid = (M + 63) / 64;
-  if (RP == 64) {
-    constexpr int smem = 3 * (64 * 64 * 2 + 64 * 64 * 2);
-    k_lora_down<64><<<grid, 128, smem, st>>>((const __nv_bfloat16*)X, (const __nv_bfloat16*)A, M,
-                                             K, r, s, (__nv_bfloat16*)sT_pad, (__nv_bfloat16*)T_save);
-  } else {
-    constexpr int smem = 3 * (64 * 64 * 2 + 128 * 64 * 2);
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_lora_down<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      attr = true;
+  if (RP == 64) launch_skinny<64, false>(X, A, M, K, r, s, sT_pad, T_save, st);
+  else launch_skinny<128, false>(X, A, M, K, r, s, sT_pad, T_save, st);
+}
+
+void launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
+                   void* sU_pad, cudaStream_t st) {
+  if (RP == 64) launch_skinny<64, true>(dY, B, M, N, r, s, sU_pad, nullptr, st);
+  else launch_skinny<128, true>(dY, B, M, N, r, s, sU_pad, nullptr, st);
+}
+
+// ===========================================================================
+// Split-M reduction products  C = P^T Q  over the token dimension:
+//   partial[chunk][TR-tile rows][TC-tile cols] = sum_{m in chunk} P[m, i] Q[m, c]
+// P is [M, Rdim] (Rdim contiguous), Q is [M, Cdim] (Cdim contiguous), both bf16.
+// dA = s U^T X uses P = sU, Q = X;  dB = s dY^T T uses P = dY, Q = T.
+// 8 warps, each 32 x 32 of the tile; operands via ldmatrix.trans.
+// ===========================================================================
+template <int TR, int TC>
+__global__ void __launch_bounds__(256)
+k_atb_partial(const __nv_bfloat16* __restrict__ P, int ldp, int Rdim,
+              const __nv_bfloat16* __restrict__ Q, int ldq, int Cdim, int M, int rows_per_chunk,
+              float* __restrict__ part, int Rpad, int Cpad) {
+  constexpr int MC = 32, STG = 3;
+  constexpr int PB = MC * TR * 2, QB = MC * TC * 2;
+  constexpr int WC = TC / 32;                       // warps along columns
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wr = warp / WC, wc = warp % WC;
+  const int i0 = blockIdx.x * TR, c0 = blockIdx.y * TC;
+  const int mbeg = blockIdx.z * rows_per_chunk;
+  const int mend = min(M, mbeg + rows_per_chunk);
+  const int nst = (mend - mbeg + MC - 1) / MC;
+
+  auto load_stage = [&](int it, int stg) {
+    uint8_t* ps = sm + stg * (PB + QB);
+    uint8_t* qs = ps + PB;
+    const int mb = mbeg + it * MC;
+    for (int c = tid; c < MC * (TR / 8); c += 256) {
+      const int row = c / (TR / 8), ch = c % (TR / 8);
+      const int m = mb + row, i = i0 + ch * 8;
+      const bool ok = m < mend && i < Rdim;
+      cp_async16(smem_u32(ps) + swzw<TR>(row, ch * 8), ok ? (const void*)(P + (int64_t)m * ldp + i) : (const void*)P,
+                 ok ? 16 : 0);
     }
-    k_lora_down<128><<<grid, 128, smem, st>>>((const __nv_bfloat16*)X, (const __nv_bfloat16*)A, M,
-                                              K, r, s, (__nv_bfloat16*)sT_pad, (__nv_bfloat16*)T_save);
+    for (int c = tid; c < MC * (TC / 8); c += 256) {
+      const int row = c / (TC / 8), ch = c % (TC / 8);
+      const int m = mb + row, cc = c0 + ch * 8;
+      const bool ok = m < mend && cc < Cdim;
+      cp_async16(smem_u32(qs) + swzw<TC>(row, ch * 8), ok ? (const void*)(Q + (int64_t)m * ldq + cc) : (const void*)Q,
+                 ok ? 16 : 0);
+    }
+  };
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = acc[a][b][2] = acc[a][b][3] = 0.f;
+
+#pragma unroll
+  for (int i = 0; i < STG - 1; ++i) {
+    if (i < nst) load_stage(i, i);
+    cp_async_commit();
   }
+  for (int it = 0; it < nst; ++it) {
+    cp_async_wait<STG - 2>();
+    __syncthreads();
+    if (it + STG - 1 < nst) load_stage(it + STG - 1, (it + STG - 1) % STG);
+    cp_async_commit();
+    const uint8_t* ps = sm + (it % STG) * (PB + QB);
+    const uint8_t* qs = ps + PB;
+#pragma unroll
+    for (int k16 = 0; k16 < MC / 16; ++k16) {
+      uint32_t af[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        // A = P^T: rows i, cols m.  Stored P[m][i]: .trans gives the fragment.
+        const int m = k16 * 16 + (lane & 7) + 8 * (lane >> 4);
+        const int i = wr * 32 + a * 16 + 8 * ((lane >> 3) & 1);
+        ldsm_x4_t(smem_u32(ps) + swzw<TR>(m, i), af[a][0], af[a][1], af[a][2], af[a][3]);
+      }
+#pragma unroll
+      for (int bp = 0; bp < 2; ++bp) {
+        // B = Q: k = m, n = c.  Stored Q[m][c]: .trans gives the fragment.
+        uint32_t b0, b1, b2, b3;
+        const int m = k16 * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int c = wc * 32 + bp * 16 + 8 * (lane >> 4);
+        ldsm_x4_t(smem_u32(qs) + swzw<TC>(m, c), b0, b1, b2, b3);
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          mma_bf16_16816(acc[a][2 * bp], af[a][0], af[a][1], af[a][2], af[a][3], b0, b1);
+          mma_bf16_16816(acc[a][2 * bp + 1], af[a][0], af[a][1], af[a][2], af[a][3], b2, b3);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  float* out = part + (int64_t)blockIdx.z * Rpad * Cpad;
+  const int g = lane >> 2, cq = (lane & 3) * 2;
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = i0 + wr * 32 + a * 16 + g + 8 * h;
+        const int c = c0 + wc * 32 + b * 8 + cq;
+        *reinterpret_cast<float2*>(out + (int64_t)i * Cpad + c) =
+            make_float2(acc[a][b][2 * h], acc[a][b][2 * h + 1]);
+      }
+}
+
+// out[i, c] = RNbf16(s * sum_{chunk = 0..n-1} part[chunk][i][c]) for i < Rdim, c < Cdim,
+// summed in chunk order (deterministic).
+__global__ void k_reduce_partials(const float* __restrict__ part, int nchunks, int Rpad, int Cpad,
+                                  int Rdim, int Cdim, float s, __nv_bfloat16* __restrict__ out) {
+  const int64_t total = (int64_t)Rdim * Cdim;
+  const int64_t plane = (int64_t)Rpad * Cpad;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / Cdim, c = e % Cdim;
+    const float* p = part + i * Cpad + c;
+    float acc = 0.f;
+    for (int k = 0; k < nchunks; ++k) acc = __fadd_rn(acc, p[k * plane]);
+    out[e] = __float2bfloat16_rn(__fmul_rn(s, acc));
+  }
+}
+
+// Split count of the token dimension: aims at ~600 CTAs whatever the device,
+// so that workspace size and summation order depend only on the shapes.
+int atb_chunks(int tiles, int M) {
+  int want = std::max(1, (600 + tiles - 1) / tiles);
+  int maxc = std::max(1, (M + 31) / 32);
+  return std::min(want, maxc);
+}
+
+// C[Rdim, Cdim] = s * P^T Q over M rows, bf16 out.  `part` must hold
+// chunks * Rpad * Cpad floats (see atb_workspace_floats).
+void launch_atb(const void* P, int ldp, int Rdim, const void* Q, int ldq, int Cdim, int M, float s,
+                void* out, float* part, int num_sms, cudaStream_t st) {
+  const bool tall = Rdim >= Cdim;                  // choose the tile shape by aspect
+  const int TR = tall ? 128 : 64, TC = tall ? 64 : 128;
+  const int gr = (Rdim + TR - 1) / TR, gc = (Cdim + TC - 1) / TC;
+  const int Rpad = gr * TR, Cpad = gc * TC;
+  const int chunks = atb_chunks(gr * gc, M);
+  const int rows_per_chunk = (((M + chunks - 1) / chunks) + 31) / 32 * 32;
+  const int nch = (M + rows_per_chunk - 1) / rows_per_chunk;
+  const dim3 grid(gr, gc, nch);
+  constexpr int smem = 3 * (32 * 128 * 2 + 32 * 64 * 2);
+  if (tall)
+    k_atb_partial<128, 64><<<grid, 256, smem, st>>>((const __nv_bfloat16*)P, ldp, Rdim,
+        (const __nv_bfloat16*)Q, ldq, Cdim, M, rows_per_chunk, part, Rpad, Cpad);
+  else
+    k_atb_partial<64, 128><<<grid, 256, smem, st>>>((const __nv_bfloat16*)P, ldp, Rdim,
+        (const __nv_bfloat16*)Q, ldq, Cdim, M, rows_per_chunk, part, Rpad, Cpad);
+  const int64_t total = (int64_t)Rdim * Cdim;
+  const int rb = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms * 8);
+  k_reduce_partials<<<std::max(rb, 1), 256, 0, st>>>(part, nch, Rpad, Cpad, Rdim, Cdim, s,
+                                                     (__nv_bfloat16*)out);
+}
+
+size_t atb_workspace_floats(int Rdim, int Cdim, int M) {
+  const bool tall = Rdim >= Cdim;
+  const int TR = tall ? 128 : 64, TC = tall ? 64 : 128;
+  const int gr = (Rdim + TR - 1) / TR, gc = (Cdim + TC - 1) / TC;
+  const int chunks = atb_chunks(gr * gc, M);
+  const int rows_per_chunk = (((M + chunks - 1) / chunks) + 31) / 32 * 32;
+  const int nch = (M + rows_per_chunk - 1) / rows_per_chunk;
+  return (size_t)nch * gr * TR * gc * TC;
+}
+
+// ===========================================================================
+// Dequantise-transpose: Wt[k, n] = deq(W)[n, k], bf16, same values as
+// nf4_dequantize.  CTA tile 64 rows (n) x 128 columns (k) = 2 NF4 blocks per
+// row; 256 threads, each dequantises 32 weights into shared memory, then the
+// tile is written out transposed with 16-byte stores.
+// ===========================================================================
+__global__ void __launch_bounds__(256)
+k_dequant_t(const uint8_t* __restrict__ packed, int N, int K, int dq,
+            const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
+            const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
+            __nv_bfloat16* __restrict__ Wt, Nf4Tables tb) {
+  __shared__ uint16_t tile[64][128 + 8];
+  __shared__ float s_q[16];
+  if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
+  __syncthreads();
+  const int n0 = blockIdx.y * 64, k0 = blockIdx.x * 128;
+  const int tid = threadIdx.x;
+  {
+    const int row = tid >> 2, part = tid & 3;        // 4 threads x 32 weights per row
+    const int n = n0 + row, k = k0 + part * 32;
+    if (n < N && k < K) {
+      const int64_t e = (int64_t)n * K + k;
+      const int64_t blk = e >> 6;
+      float a;
+      if (dq) {
+        const float c = (float)qabsmax[blk];
+        a = __fadd_rn(__fmul_rn(__fdiv_rn(c, 127.0f), dq_scale[blk >> 8]), dq_mean[0]);
+      } else {
+        a = absmax[blk];
+      }
+      const uint4 pk = *reinterpret_cast<const uint4*>(packed + (e >> 1));
+      const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t byte = (wds[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+        const uint32_t v = pack_bf16x2(__fmul_rn(s_q[byte >> 4], a), __fmul_rn(s_q[byte & 15], a));
+        tile[row][part * 32 + 2 * j] = (uint16_t)(v & 0xFFFF);
+        tile[row][part * 32 + 2 * j + 1] = (uint16_t)(v >> 16);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tile[row][part * 32 + j] = 0;
+    }
+  }
+  __syncthreads();
+  {
+    // 128 output rows (k) x 64 columns (n): 2 threads per row, 32 n each
+    const int kr = tid >> 1, half = tid & 1;
+    const int k = k0 + kr;
+    if (k < K) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int nb = half * 32 + v * 8;
+        if (n0 + nb >= N) break;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w[j] = (uint32_t)tile[nb + 2 * j][kr] | ((uint32_t)tile[nb + 2 * j + 1][kr] << 16);
+        *reinterpret_cast<uint4*>(Wt + (int64_t)k * N + n0 + nb) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
+void launch_dequant_t(const nf4_weight* w, void* Wt, cudaStream_t st) {
+  const dim3 grid((unsigned)((w->cols + 127) / 128), (unsigned)((w->rows + 63) / 64));
+  k_dequant_t<<<grid, 256, 0, st>>>(w->packed, (int)w->rows, (int)w->cols, w->double_quant,
+                                    w->absmax, w->qabsmax, w->dq_scale, w->dq_mean,
+                                    (__nv_bfloat16*)Wt, host_tables());
+}
+
+// At_pad[k, j] = A[j, k] for j < r, 0 for r <= j < RP.
+__global__ void k_transpose_pad(const __nv_bfloat16* __restrict__ A, int r, int K, int RP,
+                                __nv_bfloat16* __restrict__ At) {
+  const int64_t total = (int64_t)K * RP;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t k = e / RP;
+    const int j = (int)(e % RP);
+    At[e] = j < r ? A[(int64_t)j * K + k] : __float2bfloat16_rn(0.0f);
+  }
+}
+
+void launch_transpose_pad(const void* A, int r, int K, int RP, void* At, cudaStream_t st) {
+  const int64_t total = (int64_t)K * RP;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, 148 * 8);
+  k_transpose_pad<<<grid, 256, 0, st>>>((const __nv_bfloat16*)A, r, K, RP, (__nv_bfloat16*)At);
 }
 
 // ===========================================================================

@@ -392,6 +392,10 @@ def test_linear_fwd_bwd_vs_autograd():
     assert np.allclose(dX, X.grad.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(dA, A.grad.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(dB, B.grad.numpy(), rtol=1e-12, atol=1e-12)
+    dA2, dB2 = oracle.linear_bwd_adapters(X.detach().numpy(), dY.numpy(), A.detach().numpy(),
+                                          B.detach().numpy(), alpha, r)
+    assert np.allclose(dA2, A.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dB2, B.grad.numpy(), rtol=1e-12, atol=1e-12)
 
 
 def test_linear_special_cases():

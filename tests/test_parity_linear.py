@@ -130,3 +130,69 @@ def test_forward_mlp_7b_full_size_sampled(q):
     for which in range(3):
         W, X, A, B = synth.layer_inputs(wl, which)
         _sampled_forward(q, W, X, A, B, wl.alpha, wl.r, seed=which)
+
+
+# ---------------------------------------------------------------------------
+# Backward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,M,r,alpha,pass_T", [
+    (256, 512, 300, 16, 32.0, True),
+    (256, 512, 300, 16, 32.0, False),
+    (200, 192, 257, 8, 16.0, True),        # N not a multiple of 64: partial contraction step
+    (384, 256, 513, 64, 128.0, False),
+    (136, 320, 100, 128, 64.0, True),
+    (512, 1024, 1, 16, 32.0, False),       # decode-sized token counts
+    (512, 1024, 4, 16, 32.0, True),
+])
+def test_backward_small(q, N, K, M, r, alpha, pass_T):
+    W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=7 * M + r)
+    dY = synth.activations(M, N, 7 * M + r + 5)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    _, T = q.linear_fwd(wq, Xc, Ac, Bc, alpha)
+    dX, dA, dB = q.linear_bwd(wq, Xc, dYc, Ac, Bc, alpha, T=T if pass_T else None)
+    assert q.qlora_check_status() == 0
+    Wd = _oracle_weight(wq, W)
+    dXr, dAr, dBr = oracle.linear_bwd(X.float().numpy(), dY.float().numpy(), Wd,
+                                      A.float().numpy(), B.float().numpy(), alpha, r)
+    assert rel_err(dX, dXr) <= TOL
+    assert rel_err(dA, dAr) <= TOL
+    assert rel_err(dB, dBr) <= TOL
+
+
+def test_backward_adapter_gradients_only(q):
+    """W = 0: dX = s U A only, dA and dB unchanged by the base weight."""
+    N, K, M, r, alpha = 256, 384, 200, 32, 64.0
+    W = torch.zeros(N, K, dtype=torch.bfloat16)
+    X = synth.activations(M, K, 6001)
+    A = synth.activations(r, K, 6002, sigma=0.02)
+    B = synth.activations(N, r, 6003, sigma=0.02)
+    dY = synth.activations(M, N, 6004)
+    wq = q.quantize(W.cuda())
+    dX, dA, dB = q.linear_bwd(wq, X.cuda(), dY.cuda(), A.cuda(), B.cuda(), alpha)
+    assert q.qlora_check_status() == 0
+    dXr, dAr, dBr = oracle.linear_bwd(X.float().numpy(), dY.float().numpy(), np.zeros((N, K)),
+                                      A.float().numpy(), B.float().numpy(), alpha, r)
+    assert rel_err(dX, dXr) <= TOL and rel_err(dA, dAr) <= TOL and rel_err(dB, dBr) <= TOL
+
+
+@pytest.mark.slow
+def test_backward_4096_full_size(q):
+    """The full backward workload: dA, dB compared in full, dX on sampled rows."""
+    wl = synth.WORKLOADS["bwd_4096"]
+    W, X, A, B = synth.layer_inputs(wl, 0)
+    dY = synth.upstream_grad(wl, 0)
+    wq = q.quantize(W.cuda(), double_quant=True)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    _, T = q.linear_fwd(wq, Xc, Ac, Bc, wl.alpha)
+    dX, dA, dB = q.linear_bwd(wq, Xc, dYc, Ac, Bc, wl.alpha, T=T)
+    assert q.qlora_check_status() == 0
+    Xn, An, Bn, dYn = (t.float().numpy() for t in (X, A, B, dY))
+    dAr, dBr = oracle.linear_bwd_adapters(Xn, dYn, An, Bn, wl.alpha, wl.r)
+    assert rel_err(dA, dAr) <= TOL
+    assert rel_err(dB, dBr) <= TOL
+    rng = np.random.default_rng(4)
+    rows = np.unique(np.concatenate([rng.choice(wl.M, 48, replace=False), [0, wl.M - 1]]))
+    Wd = _oracle_weight(wq, W)
+    dXr, _, _ = oracle.linear_bwd(Xn[rows], dYn[rows], Wd, An, Bn, wl.alpha, wl.r)
+    assert rel_err(dX[rows], dXr) <= TOL
