@@ -1,0 +1,526 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 QLoRA NF4 hot path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of the 7B-class
+decoder MLP workload (gate/up W 18944x3584, down W 3584x18944, 8192 tokens,
+r=64, alpha=16), for each of the three projections:
+
+    nf4_quantize + nf4_double_quantize   (quantise the frozen bf16 weight)
+    nf4_dequantize                       (bf16 export of the base weight)
+    qlora_linear_fwd                     (fused NF4-dequant GEMM + adapter)
+    qlora_linear_bwd                     (dX, dA, dB; T saved by the forward)
+    qlora_linear_fwd at 16 tokens        (decode-sized call)
+
+Inputs are seeded synthetic Gaussians (qlora_linear_layers_b200.synth) and
+larger than L2 per step (no flush needed).  `value` is the layer's tensor
+FLOPs (forward, backward and decode of all projections, all ranks) divided
+by the device time of the step, inputs resident in HBM.  `e2e` is the same
+metric with every step's inputs copied from pinned host memory and the
+adapter gradients read back.  Under torchrun every rank runs the same
+workload on its own tokens and the adapter gradients are all-reduced
+(data-parallel; weak scaling).
+
+--impl reference times the CPU oracle (oracle/, NumPy fp64) on a bounded
+sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA NF4 linear TFLOP/s & quant/dequant GB/s, % of B200 roofline"
+WORKLOAD = "mlp_7b"
+DECODE_M = 16
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Work accounting (algorithmic FLOPs and bytes)
+# ---------------------------------------------------------------------------
+
+def layer_flops(M, N, K, r):
+    fwd = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
+    # dX = dY W' + s U A, U = dY B, dA = s U^T X, dB = s dY^T T (T saved)
+    bwd = 2 * M * N * K + 2 * M * N * r + 2 * M * K * r + 2 * M * K * r + 2 * M * N * r
+    return fwd, bwd
+
+
+def quant_bytes(n):          # read bf16, write codes + fp32 absmax
+    return n * 2 + n // 2 + 4 * (n // 64)
+
+
+def dq_bytes(n):             # read absmax twice (sum, codes), write int8 + group scales
+    na = n // 64
+    return 8 * na + na + 4 * ((na + 255) // 256)
+
+
+def dequant_bytes(n):        # read codes + int8 scales + group scales, write bf16
+    na = n // 64
+    return n // 2 + na + 4 * ((na + 255) // 256) + 2 * n
+
+
+def decode_bytes(M, N, K, r):
+    n = N * K
+    na = n // 64
+    return n // 2 + na + 4 * ((na + 255) // 256) + 2 * M * K + 2 * r * K + 2 * N * r + 2 * M * N
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_indices):
+        self.idx = ",".join(str(i) for i in gpu_indices)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.idx, "-lms", "100"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                    power.append(float(f[3]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s, p in zip(sm, power) if p > 0.5 * max(power)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power)}
+
+
+# ---------------------------------------------------------------------------
+# Our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from qlora_linear_layers_b200.build import build
+    build()
+    import qlora_linear_layers_b200 as q
+    from qlora_linear_layers_b200 import _lib, synth
+
+    lib = _lib.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[WORKLOAD]
+    M, r, alpha = wl.M, wl.r, wl.alpha
+
+    # ---- inputs: seeded on the host (pinned, for the end-to-end leg), then resident in HBM
+    host, devt = [], []
+    for p, (N, K) in enumerate(wl.weights):
+        seed_off = 100000 * rank
+        W = synth.weight(N, K, wl.seed(synth.TID_W, p) + seed_off, "bf16")
+        X = synth.activations(M, K, wl.seed(synth.TID_X, p) + seed_off)
+        A = synth.activations(r, K, wl.seed(synth.TID_A, p), sigma=0.02)
+        B = synth.activations(N, r, wl.seed(synth.TID_B, p), sigma=0.02)
+        dY = synth.activations(M, N, wl.seed(synth.TID_DY, p) + seed_off)
+        h = {k: v.pin_memory() for k, v in dict(W=W, X=X, A=A, B=B, dY=dY).items()}
+        host.append(h)
+        d = {k: v.to(dev) for k, v in h.items()}
+        n = N * K
+        na = n // 64
+        d["wq"] = q.NF4Tensor(
+            packed=torch.empty(n // 2, dtype=torch.uint8, device=dev), rows=N, cols=K,
+            absmax=torch.empty(na, dtype=torch.float32, device=dev),
+            qabsmax=torch.empty(na, dtype=torch.int8, device=dev),
+            dq_scale=torch.empty((na + 255) // 256, dtype=torch.float32, device=dev),
+            dq_mean=torch.empty(4, dtype=torch.float32, device=dev)[:1], double_quant=True)
+        d["Wdeq"] = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        d["Y"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        d["T"] = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+        d["dX"] = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        d["dA"] = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
+        d["dB"] = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+        d["Ydec"] = torch.empty(DECODE_M, N, dtype=torch.bfloat16, device=dev)
+        h["dA_out"] = torch.empty(r, K, dtype=torch.bfloat16).pin_memory()
+        h["dB_out"] = torch.empty(N, r, dtype=torch.bfloat16).pin_memory()
+        devt.append(d)
+    ws_bytes = 0
+    for (N, K) in wl.weights:
+        ws_bytes = max(ws_bytes, q.workspace_bytes(_lib.QLORA_OP_FWD, M, N, K, r),
+                       q.workspace_bytes(_lib.QLORA_OP_BWD, M, N, K, r),
+                       q.workspace_bytes(_lib.QLORA_OP_FWD, DECODE_M, N, K, r),
+                       q.workspace_bytes(_lib.QLORA_OP_DOUBLE_QUANT, 0, N * K // 64, 0, 0))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    comps = ("quantize", "double_quant", "dequantize", "fwd", "bwd", "decode")
+    stream = torch.cuda.current_stream()
+
+    def step(record, gemm_ev):
+        for p, d in enumerate(devt):
+            wq = d["wq"]
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if record is not None else None
+            if ev: ev[0].record(stream)
+            q.nf4_quantize(d["W"], wq.packed, wq.absmax)
+            if ev: ev[1].record(stream)
+            q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws)
+            if ev: ev[2].record(stream)
+            q.nf4_dequantize(wq, d["Wdeq"])
+            if ev: ev[3].record(stream)
+            if gemm_ev is not None:
+                g0, g1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                # torch creates the CUDA event on first record; the library's
+                # record at the GEMM launch supersedes this one
+                g0.record(stream)
+                g1.record(stream)
+                lib.qlora_profile_gemm_events(g0.cuda_event, g1.cuda_event)
+                gemm_ev.append((p, g0, g1))
+            q.qlora_linear_fwd(wq, d["X"], d["A"], d["B"], alpha, d["Y"], d["T"], ws)
+            if ev: ev[4].record(stream)
+            q.qlora_linear_bwd(wq, d["X"], d["dY"], d["A"], d["B"], alpha, d["dX"], d["dA"], d["dB"],
+                               T=d["T"], ws=ws)
+            if ev: ev[5].record(stream)
+            q.qlora_linear_fwd(wq, d["X"][:DECODE_M], d["A"], d["B"], alpha, d["Ydec"], None, ws)
+            if ev: ev[6].record(stream)
+            if world > 1:
+                dist.all_reduce(d["dA"])
+                dist.all_reduce(d["dB"])
+            if record is not None:
+                record.append((p, ev))
+
+    def timed(nsteps, body):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(nsteps):
+            body()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = t0.elapsed_time(t1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for _ in range(args.warmup):
+        step(None, None)
+    torch.cuda.synchronize()
+    st = q.qlora_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    rec, gemm_ev = [], []
+    sampler = ClockSampler(range(world)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    l0 = lib.qlora_kernel_launches()
+    total_ms = timed(args.steps, lambda: step(rec, gemm_ev))
+    launches = lib.qlora_kernel_launches() - l0
+    st = q.qlora_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the timed region")
+
+    # ---- accounting
+    step_flops = 0
+    fwd_fl, bwd_fl, dec_fl = [], [], []
+    for (N, K) in wl.weights:
+        f, b = layer_flops(M, N, K, r)
+        dfl, _ = layer_flops(DECODE_M, N, K, r)
+        fwd_fl.append(f); bwd_fl.append(b); dec_fl.append(dfl)
+        step_flops += f + b + dfl
+    ms_step = total_ms / args.steps
+    value = step_flops * world / (ms_step * 1e-3) / 1e12
+
+    comp_ms = {c: 0.0 for c in comps}
+    per_proj = [{c: 0.0 for c in comps} for _ in wl.weights]
+    for p, ev in rec:
+        for i, c in enumerate(comps):
+            t = ev[i].elapsed_time(ev[i + 1])
+            comp_ms[c] += t / args.steps
+            per_proj[p][c] += t / args.steps
+    gemm_ms = [0.0 for _ in wl.weights]
+    for p, g0, g1 in gemm_ev:
+        gemm_ms[p] += g0.elapsed_time(g1) / args.steps
+
+    pk = peaks()
+    hbm = pk["hbm_gbs"]
+    tc_sus = pk["bf16_tflops_sustained"]
+    tc_burst = pk["bf16_tflops"]
+    nsum = sum(N * K for (N, K) in wl.weights)
+    gbs = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9
+    components = {
+        "quantize": {"ms": comp_ms["quantize"], "GB/s": gbs(sum(quant_bytes(N * K) for N, K in wl.weights), comp_ms["quantize"])},
+        "double_quant": {"ms": comp_ms["double_quant"], "GB/s": gbs(sum(dq_bytes(N * K) for N, K in wl.weights), comp_ms["double_quant"])},
+        "dequantize": {"ms": comp_ms["dequantize"], "GB/s": gbs(sum(dequant_bytes(N * K) for N, K in wl.weights), comp_ms["dequantize"])},
+        "fwd": {"ms": comp_ms["fwd"], "TFLOP/s": sum(fwd_fl) / (comp_ms["fwd"] * 1e-3) / 1e12},
+        "bwd": {"ms": comp_ms["bwd"], "TFLOP/s": sum(bwd_fl) / (comp_ms["bwd"] * 1e-3) / 1e12},
+        "decode": {"ms": comp_ms["decode"], "GB/s": gbs(sum(decode_bytes(DECODE_M, N, K, r) for N, K in wl.weights), comp_ms["decode"])},
+    }
+    for c, v in components.items():
+        if "GB/s" in v:
+            v["frac_hbm"] = v["GB/s"] / hbm
+        else:
+            v["frac_tensor_sustained"] = v["TFLOP/s"] / tc_sus
+    components["per_projection_ms"] = per_proj
+
+    # dominant kernel: the fused NF4-dequant forward GEMM (one launch per projection)
+    gemm_flops = [2 * M * N * K + 2 * M * N * r for (N, K) in wl.weights]
+    achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    roofline = {"kernel": "k_qlora_gemm<NF4> (fused NF4-dequant forward GEMM + adapter tail)",
+                "bound": "tensor", "achieved": achieved, "peak": tc_sus, "unit": "TFLOP/s",
+                "frac": achieved / tc_sus, "traffic": None,
+                "peak_kind": f"bf16 dense, sustained ({pk['source']})",
+                "frac_of_burst_peak": achieved / tc_burst,
+                "per_launch_ms": gemm_ms,
+                "algorithmic_flops_per_launch": gemm_flops}
+
+    # ---- end-to-end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h2d = sum(h[k].numel() * h[k].element_size() for h in host for k in ("W", "X", "A", "B", "dY"))
+        d2h = sum(h[k].numel() * h[k].element_size() for h in host for k in ("dA_out", "dB_out"))
+
+        def e2e_step():
+            for h, d in zip(host, devt):
+                for k in ("W", "X", "A", "B", "dY"):
+                    d[k].copy_(h[k], non_blocking=True)
+            step(None, None)
+            for h, d in zip(host, devt):
+                h["dA_out"].copy_(d["dA"], non_blocking=True)
+                h["dB_out"].copy_(d["dB"], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e_ms = timed(args.steps, e2e_step)
+        e2e = {"value": step_flops * world / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.steps}
+        if q.qlora_check_status() != 0:
+            raise RuntimeError("device status set in the end-to-end leg")
+
+    clocks = sampler.stop() if sampler else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(budget_s=20.0)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded Gaussian, no real weights)",
+            "config": {"workload": "mlp_7b: 7B-class decoder MLP, gate/up W 18944x3584 and down "
+                                   "W 3584x18944 NF4 (block 64, DQ 256), 8192 tokens per GPU, "
+                                   "r=64, alpha=16; decode calls at 16 tokens",
+                       "tokens_per_gpu": M, "r": r, "alpha": alpha,
+                       "step": "quantize+DQ, dequantize, fwd, bwd, decode(16) per projection",
+                       "l2": "inputs larger than L2 every step (>1 GB per step); no flush",
+                       "parallelism": f"dp{world}"},
+            "e2e": e2e, "gpu_launches": int(launches),
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "components": components,
+        }
+        print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# The oracle on the host cores (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+
+def _oracle_inputs(rows, tokens):
+    """Seeded inputs of the sampled sub-layers (generation is not timed)."""
+    from qlora_linear_layers_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    out = []
+    for p, (N, K) in enumerate(wl.weights):
+        n = min(rows, N)
+        out.append(dict(
+            W=synth.weight(n, K, wl.seed(synth.TID_W, p), "bf16").float().numpy(),
+            X=synth.activations(tokens, K, wl.seed(synth.TID_X, p)).float().numpy(),
+            A=synth.activations(wl.r, K, wl.seed(synth.TID_A, p), sigma=0.02).float().numpy(),
+            B=synth.activations(n, wl.r, wl.seed(synth.TID_B, p), sigma=0.02).float().numpy(),
+            dY=synth.activations(tokens, n, wl.seed(synth.TID_DY, p)).float().numpy()))
+    return out
+
+
+def _oracle_sample(inputs):
+    """Quantise + DQ + dequantise each sampled weight (its first output rows),
+    then forward, backward and a 16-token decode of that sub-layer; returns the
+    tensor FLOPs done."""
+    import oracle
+    from qlora_linear_layers_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    flops = 0
+    for d in inputs:
+        W, X, A, B, dY = d["W"], d["X"], d["A"], d["B"], d["dY"]
+        n, K = W.shape
+        tokens = X.shape[0]
+        codes, a = oracle.quantize(W)
+        qa, s, mu = oracle.double_quantize(a)
+        Wd = oracle.dequantize(oracle.pack(codes), oracle.dq_absmax(qa, s, mu), W.shape)
+        oracle.linear_fwd(X, Wd, A, B, wl.alpha, wl.r)
+        oracle.linear_bwd(X, dY, Wd, A, B, wl.alpha, wl.r)
+        oracle.linear_fwd(X[:DECODE_M], Wd, A, B, wl.alpha, wl.r)
+        f, b = layer_flops(tokens, n, K, wl.r)
+        dd, _ = layer_flops(DECODE_M, n, K, wl.r)
+        flops += f + b + dd
+    return flops
+
+
+def _calibrate(budget_s):
+    """Sample size (rows = tokens) whose oracle pass takes about budget_s."""
+    size = 64
+    while True:
+        inp = _oracle_inputs(size, size)
+        t = time.perf_counter()
+        _oracle_sample(inp)
+        el = time.perf_counter() - t
+        if el >= budget_s / 4 or size >= 4096:
+            break
+        size *= 2
+    # cost grows between linearly and quadratically with size
+    scale = max(1.0, (budget_s / max(el, 1e-3)) ** 0.6)
+    return int(min(8192, size * scale))
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float):
+    """Time the oracle on a sample sized to roughly `budget_s` seconds."""
+    size = _calibrate(budget_s)
+    inp = _oracle_inputs(size, size)
+    t = time.perf_counter()
+    flops = _oracle_sample(inp)
+    el = time.perf_counter() - t
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"each projection cut to its first {size} output rows and {size} tokens: "
+                      "NumPy quantise + DQ + dequantise, fp64 forward, backward, 16-token decode",
+            "seconds": el}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    size = _calibrate(budget)
+    inp = _oracle_inputs(size, size)
+    for _ in range(args.warmup):
+        _oracle_sample(inp)
+    t = time.perf_counter()
+    flops = 0
+    for _ in range(args.steps):
+        flops += _oracle_sample(inp)
+    el = time.perf_counter() - t
+    value = flops / el / 1e12
+    sample = (f"each projection cut to its first {size} output rows and {size} tokens per step: "
+              "NumPy quantise + DQ + dequantise, fp64 forward, backward, 16-token decode")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Gaussian)",
+           "config": {"workload": "mlp_7b (sampled for the CPU oracle)", "parallelism": "none"},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

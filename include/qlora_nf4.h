@@ -113,6 +113,18 @@ const char* qlora_status_string(int status);
 /* ABI version of this header (major*100 + minor). */
 int qlora_abi_version(void);
 
+/* Number of kernels this library has launched in this process (all devices);
+ * a measurement aid: the difference across a region counts its launches. */
+uint64_t qlora_kernel_launches(void);
+
+/* Measurement aid.  Registers two CUDA events (cudaEvent_t, created by the
+ * caller).  The next tensor-core GEMM launch of qlora_linear_fwd or
+ * qlora_linear_bwd records `start` on its stream immediately before the GEMM
+ * kernel and `stop` immediately after it, then the registration is cleared.
+ * Passing NULL for both clears a pending registration.  Host-only, per
+ * process; returns QLORA_OK or QLORA_ERR_INVALID_ARG (exactly one NULL). */
+int qlora_profile_gemm_events(void* start, void* stop);
+
 /* ---- device entry points ---------------------------------------------- */
 
 /*

@@ -52,6 +52,8 @@ class NF4Weight(C.Structure):
 
 SIGNATURES = {
     "qlora_abi_version": (_i32, []),
+    "qlora_kernel_launches": (C.c_uint64, []),
+    "qlora_profile_gemm_events": (_i32, [_vp, _vp]),
     "qlora_status_string": (C.c_char_p, [_i32]),
     "nf4_code_table": (_i32, [C.POINTER(C.c_float)]),
     "nf4_code_thresholds": (_i32, [C.POINTER(C.c_float)]),

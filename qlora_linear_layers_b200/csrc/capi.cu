@@ -1,6 +1,7 @@
 // C ABI of libqlora_nf4.so: argument validation, workspace sizing, dispatch
 // to the sm_100a kernels, and the sticky device status word.
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -120,6 +121,19 @@ int check_weight(const nf4_weight* w) {
 
 }  // namespace
 
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static std::mutex g_ev_mu;
+static cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+
+// Take (and clear) a pending event registration.
+static void take_gemm_events(cudaEvent_t* a, cudaEvent_t* b) {
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  *a = g_ev_start; *b = g_ev_stop;
+  g_ev_start = g_ev_stop = nullptr;
+}
+
 int* device_status_ptr() {
   DeviceInfo* d = nullptr;
   return current_device(&d) == QLORA_OK ? d->status : nullptr;
@@ -132,6 +146,16 @@ using namespace qnf4;
 extern "C" {
 
 int qlora_abi_version(void) { return 100; }
+
+uint64_t qlora_kernel_launches(void) { return g_launches.load(); }
+
+int qlora_profile_gemm_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  g_ev_start = static_cast<cudaEvent_t>(start);
+  g_ev_stop = static_cast<cudaEvent_t>(stop);
+  return QLORA_OK;
+}
 
 const char* qlora_status_string(int s) {
   switch (s) {
@@ -185,7 +209,9 @@ int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols, int block
   int st = current_device(&d);
   if (st) return st;
   launch_quantize(W, dtype, rows * cols, packed, absmax, d->status, (cudaStream_t)stream, d->sms);
-  return launch_status();
+  st = launch_status();
+  if (!st) count_launches(1);
+  return st;
 }
 
 int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize, int8_t* qabsmax,
@@ -205,7 +231,9 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
   launch_double_quantize(absmax, n_absmax, qabsmax, dq_scale, dq_mean,
                          static_cast<unsigned long long*>(ws), d->status, (cudaStream_t)stream,
                          d->sms);
-  return launch_status();
+  st = launch_status();
+  if (!st) count_launches(3);
+  return st;
 }
 
 int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
@@ -217,7 +245,9 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
   st = current_device(&d);
   if (st) return st;
   launch_dequantize(w, W_out, (cudaStream_t)stream, d->sms);
-  return launch_status();
+  st = launch_status();
+  if (!st) count_launches(1);
+  return st;
 }
 
 int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
@@ -244,9 +274,11 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   void* sT = wsb + lay.sT;
   const void* Bp = B;
+  int n = 2;
   if (r < RP) {
     launch_pad_cols(B, (int)N, r, RP, wsb + lay.Bpad, s);
     Bp = wsb + lay.Bpad;
+    ++n;
   }
   launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save, s);
   GemmArgs a{};
@@ -261,9 +293,15 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   a.double_quant = w->double_quant;
   a.status = d->status;
   for (int i = 0; i < 16; ++i) a.q[i] = host_tables().q[i];
+  cudaEvent_t e0, e1;
+  take_gemm_events(&e0, &e1);
+  if (e0) cudaEventRecord(e0, s);
   st = launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
+  if (e1) cudaEventRecord(e1, s);
   if (st) return st;
-  return launch_status();
+  st = launch_status();
+  if (!st) count_launches(n);
+  return st;
 }
 
 int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
@@ -292,9 +330,11 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   void* sU = wsb + lay.sU;
   void* Wt = wsb + lay.Wt;
   void* At = wsb + lay.At;
+  int n = 9;
   if (!T) {
     launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, nullptr, Tw, s);
     T = Tw;
+    ++n;
   }
   launch_lora_u(dY, B, (int)M, (int)N, r, RP, scale, sU, s);
   launch_dequant_t(w, Wt, s);
@@ -305,14 +345,20 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   a.Mtok = (int)M; a.Nout = (int)K; a.Kc = (int)N;
   a.na = RP / 64;
   a.status = d->status;
+  cudaEvent_t e0, e1;
+  take_gemm_events(&e0, &e1);
+  if (e0) cudaEventRecord(e0, s);
   st = launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
+  if (e1) cudaEventRecord(e1, s);
   if (st) return st;
   // dA[r, K] = (s U)^T X ;  dB[N, r] = s dY^T T
   launch_atb(sU, RP, r, X, (int)K, (int)K, (int)M, 1.0f, dA, reinterpret_cast<float*>(wsb + lay.pA),
              d->sms, s);
   launch_atb(dY, (int)N, (int)N, T, r, r, (int)M, scale, dB, reinterpret_cast<float*>(wsb + lay.pB),
              d->sms, s);
-  return launch_status();
+  st = launch_status();
+  if (!st) count_launches(n);
+  return st;
 }
 
 int qlora_check_status(qlora_stream_t stream) {

@@ -20,6 +20,10 @@ __device__ __forceinline__ void set_status(int* st, int code) {
 
 int* device_status_ptr();   // host: address of the status word on the current device
 
+// Host-side launch accounting (capi.cu): count_launches(n) after every
+// successful group of n kernel launches.
+void count_launches(int n);
+
 // The 16 NF4 table values and 15 thresholds, computed on the host and passed
 // to kernels by value (they live in the kernel-parameter constant bank).
 struct Nf4Tables {
