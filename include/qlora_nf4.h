@@ -200,6 +200,36 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY,
                      void* ws, size_t ws_bytes, qlora_stream_t stream);
 
 /*
+ * Forward without a workspace argument, for callers that cannot allocate
+ * device memory: a plugin inside a host program that owns all device
+ * allocations, code running during CUDA stream capture (where cudaMalloc is
+ * not allowed), or a loop that forbids allocation after start-up.  The pages
+ * have no counterpart to this entry point; it only changes where the scratch
+ * lives.
+ *
+ * Same arguments, constraints, results and errors as qlora_linear_fwd, minus
+ * ws / ws_bytes.  Scratch is a fixed array of QLORA_FWD_NOALLOC_SCRATCH_BYTES
+ * compiled into the library; every GPU that loads the library holds it until
+ * the process exits.  Calls whose qlora_workspace_bytes(QLORA_OP_FWD, M, N, K,
+ * r) exceeds that size return QLORA_ERR_WORKSPACE before anything is enqueued
+ * (with r = 64, up to M + N = 262144 tokens plus output features).
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - No call allocates or frees memory (no cudaMalloc, cudaFree or
+ *     allocating library routine).
+ *   - All calls share the array: calls whose work overlaps on the GPU (other
+ *     streams, other host threads, the same device) race and corrupt each
+ *     other's results; order them on one stream or synchronise between them.
+ *   - Each call writes every scratch byte it reads, so nothing carries over
+ *     from the previous call.
+ */
+#define QLORA_FWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int qlora_linear_fwd_noalloc(const nf4_weight* w, const void* X, int64_t M,
+                             const void* A, const void* B, int r, float alpha,
+                             void* Y, void* T_save, qlora_stream_t stream);
+
+/*
  * Synchronise `stream`, return the sticky device status word (QLORA_OK if
  * no device-side error was recorded since the last call) and clear it.
  */

@@ -30,6 +30,8 @@ QLORA_OP_DOUBLE_QUANT = 0
 QLORA_OP_FWD = 1
 QLORA_OP_BWD = 2
 
+QLORA_FWD_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _i64, _i32, _f32, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
 
@@ -65,6 +67,8 @@ SIGNATURES = {
                                 _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i64, _vp, _vp, _i32, _f32,
                                 _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_fwd_noalloc": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
+                                        _vp, _vp, _vp]),
     "qlora_check_status": (_i32, [_vp]),
 }
 
