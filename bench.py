@@ -55,6 +55,11 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["fwd", "bwd", "quantize", "dequantize", "dq", "decode"],
+                    help="profiling aid: run one operation on one projection and exit")
+    ap.add_argument("--proj", type=int, default=0, help="--case: projection 0 gate, 1 up, 2 down")
+    ap.add_argument("--tokens", type=int, default=2048, help="--case: token count")
+    ap.add_argument("--repeat", type=int, default=3, help="--case: calls (the first warms up)")
     return ap.parse_args()
 
 
@@ -500,8 +505,59 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+def run_case(args):
+    """One operation on one projection of the workload, `--repeat` times, for
+    ncu captures of a single kernel on a small case."""
+    import torch
+    from qlora_linear_layers_b200.build import build
+    build()
+    import qlora_linear_layers_b200 as q
+    from qlora_linear_layers_b200 import _lib, synth
+    wl = synth.WORKLOADS[WORKLOAD]
+    N, K = wl.weights[args.proj]
+    M = DECODE_M if args.case == "decode" else args.tokens
+    r, alpha = wl.r, wl.alpha
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(1234 + args.proj)
+    W = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    X = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+    A = (torch.randn(r, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    B = (torch.randn(N, r, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    dY = torch.randn(M, N, device=dev, generator=g).to(torch.bfloat16)
+    wq = q.quantize(W)
+    Y, T = q.linear_fwd(wq, X, A, B, alpha)
+    Wd = torch.empty_like(W)
+    ws = torch.empty(max(q.workspace_bytes(_lib.QLORA_OP_FWD, M, N, K, r),
+                         q.workspace_bytes(_lib.QLORA_OP_BWD, M, N, K, r), 2048),
+                     dtype=torch.uint8, device=dev)
+    dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+    ops = {
+        "fwd": lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, T, ws),
+        "decode": lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, None, ws),
+        "bwd": lambda: q.qlora_linear_bwd(wq, X, dY, A, B, alpha, dX, dA, dB, T=T, ws=ws),
+        "quantize": lambda: q.nf4_quantize(W, wq.packed, wq.absmax),
+        "dq": lambda: q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws),
+        "dequantize": lambda: q.nf4_dequantize(wq, Wd),
+    }
+    torch.cuda.synchronize()
+    for i in range(args.repeat):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ops[args.case]()
+        e1.record()
+        torch.cuda.synchronize()
+        print(json.dumps({"case": args.case, "N": N, "K": K, "M": M, "call": i,
+                          "ms": e0.elapsed_time(e1)}), flush=True)
+    st = q.qlora_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
