@@ -59,7 +59,7 @@ def parse():
                     help="profiling aid: run one operation on one projection and exit")
     ap.add_argument("--proj", type=int, default=0, help="--case: projection 0 gate, 1 up, 2 down")
     ap.add_argument("--tokens", type=int, default=2048, help="--case: token count")
-    ap.add_argument("--repeat", type=int, default=3, help="--case: calls (the first warms up)")
+    ap.add_argument("--repeat", type=int, default=3, help="--case: timed calls after one warm-up call")
     return ap.parse_args()
 
 
@@ -540,14 +540,17 @@ def run_case(args):
         "dequantize": lambda: q.nf4_dequantize(wq, Wd),
     }
     torch.cuda.synchronize()
+    ops[args.case]()                                  # warm-up call
+    torch.cuda.synchronize()
+    # back-to-back calls so the host runs ahead and the events time the GPU
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
     for i in range(args.repeat):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
         ops[args.case]()
-        e1.record()
-        torch.cuda.synchronize()
-        print(json.dumps({"case": args.case, "N": N, "K": K, "M": M, "call": i,
-                          "ms": e0.elapsed_time(e1)}), flush=True)
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "N": N, "K": K, "M": M, "calls": args.repeat,
+                      "ms_per_call": e0.elapsed_time(e1) / args.repeat}), flush=True)
     st = q.qlora_check_status()
     if st != 0:
         raise RuntimeError(f"device status {st}")

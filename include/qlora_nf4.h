@@ -177,7 +177,10 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream);
  *   ws device workspace of qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r)
  * Constraints: M >= 1, N % 8 == 0, K % 64 == 0, r in {8,16,32,64,128},
  * alpha finite.  M <= 16 runs the decode (GEMV) kernel, larger M the fused
- * dequantise-in-mainloop tensor-core GEMM.
+ * dequantise-in-mainloop tensor-core GEMM.  The decode kernel applies each
+ * block's scale to that block's fp32 partial product (the table rounded to
+ * bf16 rather than each scaled weight); the GEMM uses the bf16 weights of
+ * nf4_dequantize exactly.  Both are within the layer's tolerance.
  */
 int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M,
                      const void* A, const void* B, int r, float alpha,
@@ -212,7 +215,8 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY,
  * compiled into the library; every GPU that loads the library holds it until
  * the process exits.  Calls whose qlora_workspace_bytes(QLORA_OP_FWD, M, N, K,
  * r) exceeds that size return QLORA_ERR_WORKSPACE before anything is enqueued
- * (with r = 64, up to M + N = 262144 tokens plus output features).
+ * (8192 tokens at r = 64 need about 11 MiB; with r <= 64 the limit is
+ * about 260,000 tokens, with r = 128 about 26,000).
  *   - The first call on each device resolves the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

@@ -64,16 +64,24 @@ bool valid_rank(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 
 
 int padded_rank(int r) { return r <= 64 ? 64 : 128; }
 
-// Forward workspace: sT_pad [M, RP] bf16, then Bpad [N, RP] bf16 when r < RP.
+// Forward workspace: sT_pad [M, RP] bf16, Bpad [N, RP] bf16 when r < RP,
+// then the fp32 partial sums of T = X A^T.
 struct FwdWs {
-  size_t sT, Bpad, total;
+  size_t sT, Bpad, part, gemv, total;
 };
-FwdWs fwd_ws(int64_t M, int64_t N, int r) {
+FwdWs fwd_ws(int64_t M, int64_t N, int64_t K, int r) {
   FwdWs w{};
   const int RP = padded_rank(r);
-  w.sT = 0;
-  w.Bpad = align256((size_t)M * RP * 2);
-  w.total = w.Bpad + (r < RP ? align256((size_t)N * RP * 2) : 0);
+  size_t off = 0;
+  if (M <= kDecodeMaxTokens) {   // decode path: only the GEMV's partial sums
+    w.gemv = 0;
+    w.total = align256(gemv_workspace_bytes((int)M, (int)N, (int)K, r));
+    return w;
+  }
+  w.sT = off;   off += align256((size_t)M * RP * 2);
+  w.Bpad = off; off += (r < RP ? align256((size_t)N * RP * 2) : 0);
+  w.part = off; off += align256(skinny_workspace_bytes((int)M, (int)K, RP));
+  w.total = off;
   return w;
 }
 
@@ -81,7 +89,7 @@ FwdWs fwd_ws(int64_t M, int64_t N, int r) {
 // sU [M, RP], Wt = deq(W)^T [K, N], At = A^T [K, RP] (all bf16), then the
 // fp32 split-M partial sums of dA and dB.
 struct BwdWs {
-  size_t T, sU, Wt, At, pA, pB, total;
+  size_t T, sU, Wt, At, pA, pB, pT, pU, total;
 };
 BwdWs bwd_ws(int64_t M, int64_t N, int64_t K, int r) {
   BwdWs w{};
@@ -93,6 +101,8 @@ BwdWs bwd_ws(int64_t M, int64_t N, int64_t K, int r) {
   w.At = off; off += align256((size_t)K * RP * 2);
   w.pA = off; off += align256(atb_workspace_floats(r, (int)K, (int)M) * 4);
   w.pB = off; off += align256(atb_workspace_floats((int)N, r, (int)M) * 4);
+  w.pT = off; off += align256(skinny_workspace_bytes((int)M, (int)K, RP));
+  w.pU = off; off += align256(skinny_workspace_bytes((int)M, (int)N, RP));
   w.total = off;
   return w;
 }
@@ -190,7 +200,8 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     case QLORA_OP_DOUBLE_QUANT: return 256 * sizeof(unsigned long long);
     case QLORA_OP_FWD:
       if (M < 1 || N < 1 || !valid_rank(r)) return 0;
-      return fwd_ws(M, N, r).total;
+      if (K < 1) return 0;
+      return fwd_ws(M, N, K, r).total;
     case QLORA_OP_BWD:
       if (M < 1 || N < 1 || K < 1 || !valid_rank(r)) return 0;
       return bwd_ws(M, N, K, r).total;
@@ -262,7 +273,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
       (T_save && !aligned16(T_save)))
     return QLORA_ERR_ALIGN;
-  const FwdWs lay = fwd_ws(M, N, r);
+  const FwdWs lay = fwd_ws(M, N, K, r);
   if (!ws || ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   DeviceInfo* d = nullptr;
@@ -272,15 +283,25 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   const int RP = padded_rank(r);
   const float scale = alpha / (float)r;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  if (M <= kDecodeMaxTokens) {
+    // decode-sized call: HBM-bound GEMV on the warp-level tensor cores
+    const int n = launch_qlora_gemv(w, X, (int)M, A, B, r, scale, Y, T_save,
+                                    reinterpret_cast<float*>(wsb + lay.gemv), host_tables().q, s,
+                                    d->sms);
+    st = launch_status();
+    if (!st) count_launches(n);
+    return st;
+  }
   void* sT = wsb + lay.sT;
   const void* Bp = B;
-  int n = 2;
+  int n = 1;
   if (r < RP) {
     launch_pad_cols(B, (int)N, r, RP, wsb + lay.Bpad, s);
     Bp = wsb + lay.Bpad;
     ++n;
   }
-  launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save, s);
+  n += launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save,
+                        reinterpret_cast<float*>(wsb + lay.part), s);
   GemmArgs a{};
   a.packed = w->packed;
   a.absmax = w->absmax;
@@ -288,6 +309,8 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   a.dq_scale = w->dq_scale;
   a.dq_mean = w->dq_mean;
   a.out = static_cast<__nv_bfloat16*>(Y);
+  a.wad = static_cast<const __nv_bfloat16*>(Bp);
+  a.RP = RP;
   a.Mtok = (int)M; a.Nout = (int)N; a.Kc = (int)K;
   a.na = RP / 64;
   a.double_quant = w->double_quant;
@@ -330,18 +353,20 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   void* sU = wsb + lay.sU;
   void* Wt = wsb + lay.Wt;
   void* At = wsb + lay.At;
-  int n = 9;
+  int n = 7;   // dequant_t, transpose_pad, GEMM, 2 x (partials + reduce)
   if (!T) {
-    launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, nullptr, Tw, s);
+    n += launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, nullptr, Tw,
+                          reinterpret_cast<float*>(wsb + lay.pT), s);
     T = Tw;
-    ++n;
   }
-  launch_lora_u(dY, B, (int)M, (int)N, r, RP, scale, sU, s);
+  n += launch_lora_u(dY, B, (int)M, (int)N, r, RP, scale, sU, reinterpret_cast<float*>(wsb + lay.pU), s);
   launch_dequant_t(w, Wt, s);
   launch_transpose_pad(A, r, (int)K, RP, At, s);
   // dX[M, K] = dY Wt^T + sU At^T   (tokens = dY rows, outputs = K, contraction = N)
   GemmArgs a{};
   a.out = static_cast<__nv_bfloat16*>(dX);
+  a.wad = static_cast<const __nv_bfloat16*>(At);
+  a.RP = RP;
   a.Mtok = (int)M; a.Nout = (int)K; a.Kc = (int)N;
   a.na = RP / 64;
   a.status = d->status;

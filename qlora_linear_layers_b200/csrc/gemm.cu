@@ -25,10 +25,12 @@
 // accumulator, with the rank padded to 64 by zeros.
 //
 // Persistent: one CTA per SM walks a static tile schedule.  Warp 0 issues
-// TMA, warp 1 issues MMA, warps 2-9 drain the accumulator (two warps per TMEM
-// lane quadrant, 128 columns each), warps 10-13 convert NF4 (MODE_NF4).  The
-// accumulator is released as soon as it sits in registers, so the next tile's
-// MMAs overlap the stores.  Every wait is bounded (status QLORA_ERR_TIMEOUT).
+// TMA, warp 1 issues MMA, warps 2-5 drain the accumulator (one per TMEM lane
+// quadrant, in two halves of 128 columns; the accumulator is released once the
+// second half sits in registers, so the next tile's MMAs overlap the stores),
+// warps 6-13 convert NF4 (MODE_NF4): two warps per quadrant take alternate K
+// steps, so one warp's TMEM-store wait and barrier hand-off overlap the other's
+// table expansion.  Every wait is bounded (status QLORA_ERR_TIMEOUT).
 
 #include <algorithm>
 #include <cstdint>
@@ -46,25 +48,28 @@ namespace eng {
 constexpr int BN = 128;          // weight-side rows per tile (MMA M)
 constexpr int BM = 256;          // tokens per tile (MMA N)
 constexpr int BK = 64;           // contraction per stage (= one NF4 block)
-constexpr int STAGES = 4;
 constexpr int MAX_NA = 2;        // adapter K steps (r <= 128)
 constexpr int X_BYTES = BM * BK * 2;            // 32 KB token tile
 constexpr int W_BYTES = BN * BK * 2;            // 16 KB weight tile
 constexpr int ACC_COL = 0;                      // accumulator: TMEM columns [0, 256)
-constexpr int A_COL = 256;                      // NF4 A ring: STAGES x 32 columns
+constexpr int A_COL = 256;                      // NF4 A ring: stages x 32 columns
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 448;                // 14 warps
-constexpr int EPI_WARP0 = 2;
-constexpr int CVT_WARP0 = 10;
+constexpr int EPI_WARP0 = 2;                    // warps 2-5: epilogue
+constexpr int CVT_WARP0 = 6;                    // warps 6-13: converters
+
+// Pipeline depth.  MODE_NF4 keeps only token tiles in shared memory (the
+// weight side lives in TMEM), so it affords 6 stages of 32 KB; MODE_BF16 holds
+// a 16 KB weight tile beside each token tile and keeps 4.
+template <int MODE> __host__ __device__ constexpr int stages() { return MODE == MODE_NF4 ? 6 : 4; }
 
 template <int MODE>
 struct Smem {
-  uint8_t x[STAGES][X_BYTES];
-  // MODE_NF4: adapter weight tiles;  MODE_BF16: weight tile of each stage
-  uint8_t w[MODE == MODE_NF4 ? MAX_NA : STAGES][W_BYTES];
-  uint64_t x_full[STAGES], x_empty[STAGES];
-  uint64_t a_full[STAGES], a_empty[STAGES];
-  uint64_t aux_full[MAX_NA], aux_empty[MAX_NA];
+  static constexpr int NS = stages<MODE>();
+  uint8_t x[NS][X_BYTES];
+  uint8_t w[MODE == MODE_NF4 ? 1 : NS][MODE == MODE_NF4 ? 16 : W_BYTES];
+  uint64_t x_full[NS], x_empty[NS];
+  uint64_t a_full[NS], a_empty[NS];
   uint64_t acc_full, acc_empty, done;
   uint32_t tmem_base;
   int abort;
@@ -132,16 +137,18 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
   const int nk = (p.Kc + BK - 1) / BK;
   const int na = p.na;
 
+  constexpr int NS = stages<MODE>();
+  const int nsteps = nk + na;                      // ring steps per tile
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&S.x_full[i], 1);
       mbar_init(&S.x_empty[i], 1);
       mbar_init(&S.a_full[i], 128);
       mbar_init(&S.a_empty[i], 1);
     }
-    for (int i = 0; i < MAX_NA; ++i) { mbar_init(&S.aux_full[i], 1); mbar_init(&S.aux_empty[i], 1); }
     mbar_init(&S.acc_full, 1);
-    mbar_init(&S.acc_empty, 256);
+    mbar_init(&S.acc_empty, 128);
     mbar_init(&S.done, 1);
     S.abort = 0;
     mbar_fence_init();
@@ -155,8 +162,10 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_tok);
     tma_prefetch_desc(&tm_tokad);
-    tma_prefetch_desc(&tm_wad);
-    if (MODE == MODE_BF16) tma_prefetch_desc(&tm_w);
+    if (MODE == MODE_BF16) {
+      tma_prefetch_desc(&tm_wad);
+      tma_prefetch_desc(&tm_w);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -166,35 +175,27 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Step ks < nk: token tile of contraction block ks (and, MODE_BF16, the
+    // weight tile); ks >= nk: adapter step j = ks - nk (s*T or s*U tile, and,
+    // MODE_BF16, the adapter weight tile).
     if (lane == 0) {
-      uint32_t xi = 0, lt = 0;
+      uint32_t xi = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
         const int n0 = (tile % n_tiles_n) * BN;
         const int m0 = (tile / n_tiles_n) * BM;
-        for (int ks = 0; ks < nk + na; ++ks, ++xi) {
-          const int s = xi % STAGES;
-          if (!(ok = mbar_wait(&S.x_empty[s], ((xi / STAGES) & 1) ^ 1, abort, p.status))) break;
+        for (int ks = 0; ks < nsteps; ++ks, ++xi) {
+          const int s = xi % NS;
+          if (!(ok = mbar_wait(&S.x_empty[s], ((xi / NS) & 1) ^ 1, abort, p.status))) break;
+          const bool ad = ks >= nk;
+          const int kc = (ad ? ks - nk : ks) * BK;
           if (MODE == MODE_BF16) {
             mbar_arrive_expect_tx(&S.x_full[s], X_BYTES + W_BYTES);
-            if (ks < nk) {
-              tma_load_2d(S.x[s], &tm_tok, &S.x_full[s], ks * BK, m0);
-              tma_load_2d(S.w[s], &tm_w, &S.x_full[s], ks * BK, n0);
-            } else {
-              tma_load_2d(S.x[s], &tm_tokad, &S.x_full[s], (ks - nk) * BK, m0);
-              tma_load_2d(S.w[s], &tm_wad, &S.x_full[s], (ks - nk) * BK, n0);
-            }
+            tma_load_2d(S.x[s], ad ? &tm_tokad : &tm_tok, &S.x_full[s], kc, m0);
+            tma_load_2d(S.w[s], ad ? &tm_wad : &tm_w, &S.x_full[s], kc, n0);
           } else {
             mbar_arrive_expect_tx(&S.x_full[s], X_BYTES);
-            if (ks < nk) {
-              tma_load_2d(S.x[s], &tm_tok, &S.x_full[s], ks * BK, m0);
-            } else {
-              const int j = ks - nk;
-              tma_load_2d(S.x[s], &tm_tokad, &S.x_full[s], j * BK, m0);
-              if (!(ok = mbar_wait(&S.aux_empty[j], (lt & 1) ^ 1, abort, p.status))) break;
-              mbar_arrive_expect_tx(&S.aux_full[j], W_BYTES);
-              tma_load_2d(S.w[j], &tm_wad, &S.aux_full[j], j * BK, n0);
-            }
+            tma_load_2d(S.x[s], ad ? &tm_tokad : &tm_tok, &S.x_full[s], kc, m0);
           }
         }
       }
@@ -203,32 +204,28 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(BN, BM);
-      uint32_t xi = 0, ai = 0, lt = 0;
+      uint32_t xi = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++lt) {
         ok = mbar_wait(&S.acc_empty, (lt & 1) ^ 1, abort, p.status);
         if (!ok) break;
         tc_fence_after();
-        for (int ks = 0; ks < nk && ok; ++ks, ++xi) {
-          const int s = xi % STAGES;
+        for (int ks = 0; ks < nsteps && ok; ++ks, ++xi) {
+          const int s = xi % NS;
+          const uint32_t par = (xi / NS) & 1;
+          ok = mbar_wait(&S.x_full[s], par, abort, p.status);
+          if (ok && MODE == MODE_NF4) ok = mbar_wait(&S.a_full[s], par, abort, p.status);
+          if (!ok) break;
+          tc_fence_after();
           const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
           if (MODE == MODE_NF4) {
-            const int sa = ai % STAGES;
-            ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status) &&
-                 mbar_wait(&S.a_full[sa], (ai / STAGES) & 1, abort, p.status);
-            if (!ok) break;
-            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              mma_ts(tmem + ACC_COL, tmem + A_COL + sa * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
+              mma_ts(tmem + ACC_COL, tmem + A_COL + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
                      idesc, (ks > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&S.x_empty[s]);
-            mma_commit(&S.a_empty[sa]);
-            ++ai;
+            mma_commit(&S.a_empty[s]);
           } else {
-            ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status);
-            if (!ok) break;
-            tc_fence_after();
             const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[s]));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
@@ -237,20 +234,6 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
             mma_commit(&S.x_empty[s]);
           }
         }
-        for (int j = 0; j < na && ok; ++j, ++xi) {
-          const int s = xi % STAGES;
-          ok = mbar_wait(&S.x_full[s], (xi / STAGES) & 1, abort, p.status);
-          if (ok && MODE == MODE_NF4) ok = mbar_wait(&S.aux_full[j], lt & 1, abort, p.status);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[MODE == MODE_NF4 ? j : s]));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ss(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, 1u);
-          mma_commit(&S.x_empty[s]);
-          if (MODE == MODE_NF4) mma_commit(&S.aux_empty[j]);
-        }
         if (ok) mma_commit(&S.acc_full);
       }
       // all MMAs issued by this thread are complete once `done` flips
@@ -258,105 +241,126 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
       mbar_wait(&S.done, 0, abort, p.status);
     }
   } else if (warp >= CVT_WARP0) {
-    // ------------------------------------------------------------ NF4 -> bf16 converters
+    // ------------------------------------------------------------ A-operand producers (TMEM)
+    // MODE_NF4 only.  Step ks < nk: NF4 -> bf16 for block ks of the thread's
+    // weight row; step ks >= nk: copy 64 bf16 of the row's adapter factor
+    // B[n, j*64 .. j*64+63] (zero-padded to RP columns).
     if (MODE == MODE_NF4) {
       const int quad = warp & 3;
+      const uint32_t par = (uint32_t)((warp - CVT_WARP0) >> 2);   // steps of this parity
       const int row_in_tile = quad * 32 + lane;
       const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
       const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
       const int64_t kb_per_row = p.Kc / 64;
-      uint32_t ai = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      // ring step ai is step (ai % nsteps) of this CTA's tile (ai / nsteps)
+      struct Src { uint4 c[8]; float a_raw, sg; int qa; bool valid, ad; };
+      auto fetch = [&](uint32_t ai, Src& d) -> bool {
+        const uint32_t lt = ai / (uint32_t)nsteps;
+        const int ks = (int)(ai - lt * (uint32_t)nsteps);
+        const int tile = blockIdx.x + (int)lt * gridDim.x;
+        if (tile >= n_tiles) return false;
         const int n = (tile % n_tiles_n) * BN + row_in_tile;
-        const bool valid = n < p.Nout;
-        const uint4* codes =
-            reinterpret_cast<const uint4*>(p.packed + (int64_t)(valid ? n : 0) * (p.Kc / 2));
-        const int64_t blk0 = (int64_t)(valid ? n : 0) * kb_per_row;
-        // software pipeline: data for step ks+1 is loaded while step ks converts
-        uint4 c0 = __ldcg(codes), c1 = __ldcg(codes + 1);
-        float a_raw = 0.0f;
-        int qa = 0;
-        if (DQ) qa = __ldcg(p.qabsmax + blk0); else a_raw = __ldcg(p.absmax + blk0);
-        float sg = DQ ? __ldg(p.dq_scale + (blk0 >> 8)) : 0.0f;
-        for (int ks = 0; ks < nk; ++ks, ++ai) {
-          uint4 n0v = c0, n1v = c1;
-          int nqa = qa;
-          float na_raw = a_raw, nsg = sg;
-          if (ks + 1 < nk) {
-            n0v = __ldcg(codes + 2 * (ks + 1));
-            n1v = __ldcg(codes + 2 * (ks + 1) + 1);
-            const int64_t b = blk0 + ks + 1;
-            if (DQ) { nqa = __ldcg(p.qabsmax + b); nsg = __ldg(p.dq_scale + (b >> 8)); }
-            else na_raw = __ldcg(p.absmax + b);
-          }
-          // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
-          const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[qa + 127], sg), mu) : a_raw;
-          uint32_t v[32];
-          if (valid) {
-            const Lut l = build_lut(a, p.q);
-            const uint32_t wds[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        d.valid = n < p.Nout;
+        d.ad = ks >= nk;
+        const int64_t nn = d.valid ? n : 0;
+        if (d.ad) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.wad + nn * p.RP + (ks - nk) * BK);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
-          const int sa = ai % STAGES;
-          if (!mbar_wait(&S.a_empty[sa], ((ai / STAGES) & 1) ^ 1, abort, p.status)) { ok = false; break; }
-          __syncwarp();
-          tc_fence_after();
-          const uint32_t taddr = tmem + tmem_lane + A_COL + sa * 32;
-          tmem_st16(taddr, v);
-          tmem_st16(taddr + 16, v + 16);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&S.a_full[sa]);
-          c0 = n0v; c1 = n1v; qa = nqa; a_raw = na_raw; sg = nsg;
+          for (int i = 0; i < 8; ++i) d.c[i] = __ldcg(src + i);
+        } else {
+          const uint4* codes = reinterpret_cast<const uint4*>(p.packed + nn * (p.Kc / 2)) + 2 * ks;
+          d.c[0] = __ldcg(codes);
+          d.c[1] = __ldcg(codes + 1);
+          const int64_t b = nn * kb_per_row + ks;
+          if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); d.a_raw = 0.f; }
+          else { d.a_raw = __ldcg(p.absmax + b); d.qa = 0; d.sg = 0.f; }
         }
+        return true;
+      };
+      Src cur, nxt;
+      uint32_t ai = par;
+      bool have = fetch(ai, cur);
+      while (have) {
+        const bool more = fetch(ai + 2, nxt);     // prefetch this warp's next step
+        uint32_t v[32];
+        if (!cur.valid) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        } else if (cur.ad) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] = cur.c[i].x; v[4 * i + 1] = cur.c[i].y;
+            v[4 * i + 2] = cur.c[i].z; v[4 * i + 3] = cur.c[i].w;
+          }
+        } else {
+          // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
+          const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 127], cur.sg), mu) : cur.a_raw;
+          const Lut l = build_lut(a, p.q);
+          const uint32_t wds[8] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w,
+                                   cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
+        }
+        const int sa = ai % NS;
+        if (!mbar_wait(&S.a_empty[sa], ((ai / NS) & 1) ^ 1, abort, p.status)) break;
+        __syncwarp();
+        tc_fence_after();
+        const uint32_t taddr = tmem + tmem_lane + A_COL + sa * 32;
+        tmem_st16(taddr, v);
+        tmem_st16(taddr + 16, v + 16);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&S.a_full[sa]);
+        cur = nxt;
+        have = more;
+        ai += 2;
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
-    constexpr int COLS = BM / 2;                 // accumulator columns per epilogue warp
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    constexpr int HALF = BM / 2;                 // columns drained per round
     const int quad = warp & 3;
-    const int col0 = ((warp - EPI_WARP0) >> 2) * COLS;
     const int row_in_tile = quad * 32 + lane;
     const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
+    const bool odd = lane & 1;
     uint32_t lt = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++lt) {
       const int n0 = (tile % n_tiles_n) * BN;
-      const int m0 = (tile / n_tiles_n) * BM + col0;
+      const int mt = (tile / n_tiles_n) * BM;
       if (!mbar_wait(&S.acc_full, lt & 1, abort, p.status)) break;
       __syncwarp();
       tc_fence_after();
-      uint32_t packed[COLS / 2];
-#pragma unroll
-      for (int c = 0; c < COLS; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + tmem_lane + ACC_COL + col0 + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          packed[c / 2 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-      }
-      tc_fence_before();
-      mbar_arrive(&S.acc_empty);
       // lane pairs (o, o+1) swap halves so each lane stores two adjacent
       // outputs of one token row: even lanes row m, odd lanes row m+1
-      const bool odd = lane & 1;
       const int ocol = n0 + row_in_tile - (odd ? 1 : 0);
-      const int mfirst = m0 + (odd ? 1 : 0);
-      const int rows_left = (ocol < p.Nout) ? p.Mtok - mfirst : 0;
-      uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (int64_t)mfirst * p.Nout + ocol);
       const int step = p.Nout;                   // two bf16 rows = Nout words
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t packed[HALF / 2];
 #pragma unroll
-      for (int c = 0; c < COLS; c += 2) {
-        const uint32_t mine = packed[c / 2];
-        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-        const uint32_t out = odd ? prmt(other, mine, 0x7632) : prmt(mine, other, 0x5410);
-        if (c < rows_left) *dst = out;
-        dst += step;
+        for (int c = 0; c < HALF; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + tmem_lane + ACC_COL + h * HALF + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            packed[c / 2 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        }
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(&S.acc_empty);
+        }
+        const int mfirst = mt + h * HALF + (odd ? 1 : 0);
+        const int rows_left = (ocol < p.Nout) ? p.Mtok - mfirst : 0;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (int64_t)mfirst * p.Nout + ocol);
+#pragma unroll
+        for (int c = 0; c < HALF; c += 2) {
+          const uint32_t mine = packed[c / 2];
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          const uint32_t out = odd ? prmt(other, mine, 0x7632) : prmt(mine, other, 0x5410);
+          if (c < rows_left) *dst = out;
+          dst += step;
+        }
       }
     }
   }

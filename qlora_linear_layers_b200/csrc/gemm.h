@@ -21,6 +21,8 @@ struct GemmArgs {
   const int8_t* qabsmax;      // [Nout*Kc/64]     (double_quant == 1)
   const float* dq_scale;      // [ceil(Nout*Kc/64/256)]
   const float* dq_mean;       // [1]
+  const __nv_bfloat16* wad;   // [Nout, RP] adapter weight factor (MODE_NF4 reads it directly)
+  int RP;                     // adapter width padded to a multiple of 64
   __nv_bfloat16* out;         // [Mtok, Nout]
   int Mtok, Nout, Kc;
   int na;                     // adapter K steps = RP / 64
@@ -33,19 +35,31 @@ struct GemmArgs {
 int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* tokad,
                       const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);
 
+// Decode-sized forward (M <= 16): Y = X deq(W)^T + s (X A^T) B^T, T_save =
+// RNbf16(X A^T) when not null.  `part` holds gemv_workspace_bytes(M, N, K, r)
+// bytes.  Returns the number of kernels launched.
+constexpr int kDecodeMaxTokens = 16;
+int launch_qlora_gemv(const nf4_weight* w, const void* X, int M, const void* A, const void* B,
+                      int r, float s, void* Y, void* T_save, float* part, const float* q,
+                      cudaStream_t st, int num_sms);
+size_t gemv_workspace_bytes(int M, int N, int K, int r);
+
 // 2-D bf16 tensor map, 128-byte swizzle, box [box_outer rows x box_inner cols].
 bool make_tmap_2d_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer);
 
 // T = X A^T on tensor cores (mma.sync), written as
-//   sT_pad[M, RP] = RNbf16(s * T)  (zero for columns >= r)
+//   sT_pad[M, RP] = RNbf16(s * T)  (zero for columns >= r; may be null)
 //   T_save[M, r]  = RNbf16(T)      (if not null)
-void launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
-                      void* sT_pad, void* T_save, cudaStream_t st);
+// `part` holds skinny_workspace_bytes(M, K, RP) bytes of fp32 partial sums.
+// Returns the number of kernels launched.
+int launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
+                     void* sT_pad, void* T_save, float* part, cudaStream_t st);
+size_t skinny_workspace_bytes(int M, int L, int RP);
 
 // U = dY B:  sU_pad[M, RP] = RNbf16(s * U), zero beyond r.
-void launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
-                   void* sU_pad, cudaStream_t st);
+int launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
+                  void* sU_pad, float* part, cudaStream_t st);
 
 // C[Rdim, Cdim] = RNbf16(s * P^T Q) over M token rows, split over the tokens
 // into fixed chunks summed in order; `part` holds atb_workspace_floats floats.

@@ -59,24 +59,31 @@ __device__ __forceinline__ uint32_t swzw(int row, int col) {
 // Skinny product  S[M, RP] = Z[M, L] * R   (R = A^T or B; rank <= 128)
 //   BT = false: R[l, j] = A[j, l]   (A is [r, L], L contiguous)   -> T = X A^T
 //   BT = true : R[l, j] = B[l, j]   (B is [L, r], r contiguous)   -> U = dY B
-// CTA = 64 rows of Z x RP columns, 4 warps x 16 rows, L in chunks of 64.
-// Outputs: Ss[M, RP] = RNbf16(s * S) (zero beyond r), Sraw[M, r] = RNbf16(S).
+// CTA = 128 rows of Z x RP columns (8 warps x 16 rows) over one slice of the
+// contraction (blockIdx.y of `splits`), so that small token counts still
+// spread over the GPU.  One slice: the CTA writes
+//   Ss[M, RP] = RNbf16(s * S) (zero beyond r), Sraw[M, r] = RNbf16(S);
+// several: fp32 partials part[split][M][RP], summed in order by
+// k_skinny_reduce.
 // ===========================================================================
 template <int RP, bool BT>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restrict__ R, int M,
-              int L, int r, float s, __nv_bfloat16* __restrict__ Ss, __nv_bfloat16* __restrict__ Sraw) {
-  constexpr int TM = 64, KC = 64, STG = 3;
+              int L, int r, float s, int chunks_per_split, __nv_bfloat16* __restrict__ Ss,
+              __nv_bfloat16* __restrict__ Sraw, float* __restrict__ part) {
+  constexpr int TM = 128, KC = 64, STG = 3;
   constexpr int XB = TM * KC * 2, AB = RP * KC * 2;
   extern __shared__ __align__(128) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * TM;
-  const int nkc = (L + KC - 1) / KC;
+  const int nkc_all = (L + KC - 1) / KC;
+  const int kc0 = blockIdx.y * chunks_per_split;
+  const int nkc = min(nkc_all - kc0, chunks_per_split);
 
   auto load_stage = [&](int kc, int stg) {
     uint8_t* xs = sm + stg * (XB + AB);
     uint8_t* as = xs + XB;
-    for (int c = tid; c < TM * 8; c += 128) {
+    for (int c = tid; c < TM * 8; c += 256) {
       const int row = c >> 3, ch = c & 7;
       const int m = m0 + row, l = kc * KC + ch * 8;
       const bool ok = m < M && l < L;
@@ -84,7 +91,7 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
                  ok ? 16 : 0);
     }
     if (!BT) {
-      for (int c = tid; c < RP * 8; c += 128) {
+      for (int c = tid; c < RP * 8; c += 256) {
         const int row = c >> 3, ch = c & 7;            // row = j, chunk along l
         const int l = kc * KC + ch * 8;
         const bool ok = row < r && l < L;
@@ -92,7 +99,7 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
                    ok ? 16 : 0);
       }
     } else {
-      for (int c = tid; c < KC * (RP / 8); c += 128) {
+      for (int c = tid; c < KC * (RP / 8); c += 256) {
         const int row = c / (RP / 8), ch = c % (RP / 8);   // row = l, chunk along j
         const int l = kc * KC + row;
         const bool ok = l < L && ch * 8 < r;
@@ -108,13 +115,13 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
 
 #pragma unroll
   for (int i = 0; i < STG - 1; ++i) {
-    if (i < nkc) load_stage(i, i);
+    if (i < nkc) load_stage(kc0 + i, i);
     cp_async_commit();
   }
   for (int kc = 0; kc < nkc; ++kc) {
     cp_async_wait<STG - 2>();
     __syncthreads();
-    if (kc + STG - 1 < nkc) load_stage(kc + STG - 1, (kc + STG - 1) % STG);
+    if (kc + STG - 1 < nkc) load_stage(kc0 + kc + STG - 1, (kc + STG - 1) % STG);
     cp_async_commit();
     const uint8_t* xs = sm + (kc % STG) * (XB + AB);
     const uint8_t* as = xs + XB;
@@ -146,6 +153,7 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
   cp_async_wait<0>();
 
   const int g = lane >> 2, c2 = (lane & 3) * 2;
+  const bool direct = gridDim.y == 1;
 #pragma unroll
   for (int t = 0; t < RP / 8; ++t) {
     const int col = t * 8 + c2;
@@ -154,6 +162,10 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
       const int m = m0 + warp * 16 + g + 8 * h;
       if (m >= M) continue;
       const float v0 = acc[t][2 * h], v1 = acc[t][2 * h + 1];
+      if (!direct) {
+        *reinterpret_cast<float2*>(part + ((int64_t)blockIdx.y * M + m) * RP + col) = make_float2(v0, v1);
+        continue;
+      }
       if (Ss)
         *reinterpret_cast<uint32_t*>(Ss + (int64_t)m * RP + col) =
             pack_bf16x2(__fmul_rn(s, v0), __fmul_rn(s, v1));
@@ -163,30 +175,80 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
   }
 }
 
+// Sum the contraction slices in order and write Ss / Sraw as above.
+__global__ void k_skinny_reduce(const float* __restrict__ part, int splits, int M, int RP, int r,
+                                float s, __nv_bfloat16* __restrict__ Ss, __nv_bfloat16* __restrict__ Sraw) {
+  const int64_t total = (int64_t)M * RP / 2;
+  const int64_t plane = (int64_t)M * RP;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = 2 * e;
+    float a0 = 0.f, a1 = 0.f;
+    for (int k = 0; k < splits; ++k) {
+      const float2 v = *reinterpret_cast<const float2*>(part + k * plane + i);
+      a0 = __fadd_rn(a0, v.x);
+      a1 = __fadd_rn(a1, v.y);
+    }
+    const int64_t m = i / RP;
+    const int col = (int)(i % RP);
+    if (Ss) *reinterpret_cast<uint32_t*>(Ss + i) = pack_bf16x2(__fmul_rn(s, a0), __fmul_rn(s, a1));
+    if (Sraw && col < r) *reinterpret_cast<uint32_t*>(Sraw + m * r + col) = pack_bf16x2(a0, a1);
+  }
+}
+
+// Number of contraction slices for an M x L skinny product: enough CTAs to
+// cover the GPU twice over (~296), whatever the device, so that the workspace
+// size and summation order depend only on the shapes.
+int skinny_splits(int M, int L) {
+  const int tiles = (M + 127) / 128;
+  const int nkc = (L + 63) / 64;
+  int splits = std::min(std::max(1, (296 + tiles - 1) / tiles), nkc);
+  const int cps = (nkc + splits - 1) / splits;
+  return (nkc + cps - 1) / cps;
+}
+
+size_t skinny_workspace_bytes(int M, int L, int RP) {
+  const int sp = skinny_splits(M, L);
+  return sp > 1 ? (size_t)sp * M * RP * 4 : 0;
+}
+
 template <int RP, bool BT>
 static void launch_skinny(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
-                          void* Sraw, cudaStream_t st) {
-  constexpr int smem = 3 * (64 * 64 * 2 + RP * 64 * 2);
+                          void* Sraw, float* part, cudaStream_t st) {
+  constexpr int smem = 3 * (128 * 64 * 2 + RP * 64 * 2);
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(k_lora_skinny<RP, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     attr = true;
   }
-  k_lora_skinny<RP, BT><<<(M + 63) / 64, 128, smem, st>>>(
-      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)R, M, L, r, s, (__nv_bfloat16*)Ss,
-      (__nv_bfloat16*)Sraw);
+  const int splits = skinny_splits(M, L);
+  const int nkc = (L + 63) / 64;
+  const int cps = (nkc + splits - 1) / splits;
+  const dim3 grid((M + 127) / 128, splits);
+  k_lora_skinny<RP, BT><<<grid, 256, smem, st>>>(
+      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)R, M, L, r, s, cps, (__nv_bfloat16*)Ss,
+      (__nv_bfloat16*)Sraw, part);
+  if (splits > 1) {
+    const int64_t total = (int64_t)M * RP / 2;
+    const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 8);
+    k_skinny_reduce<<<blocks, 256, 0, st>>>(part, splits, M, RP, r, s, (__nv_bfloat16*)Ss,
+                                            (__nv_bfloat16*)Sraw);
+  }
 }
 
-void launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
-                      void* sT_pad, void* T_save, cudaStream_t st) {
-  if (RP == 64) launch_skinny<64, false>(X, A, M, K, r, s, sT_pad, T_save, st);
-  else launch_skinny<128, false>(X, A, M, K, r, s, sT_pad, T_save, st);
+// Returns the number of kernels launched.
+int launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
+                     void* sT_pad, void* T_save, float* part, cudaStream_t st) {
+  if (RP == 64) launch_skinny<64, false>(X, A, M, K, r, s, sT_pad, T_save, part, st);
+  else launch_skinny<128, false>(X, A, M, K, r, s, sT_pad, T_save, part, st);
+  return skinny_splits(M, K) > 1 ? 2 : 1;
 }
 
-void launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
-                   void* sU_pad, cudaStream_t st) {
-  if (RP == 64) launch_skinny<64, true>(dY, B, M, N, r, s, sU_pad, nullptr, st);
-  else launch_skinny<128, true>(dY, B, M, N, r, s, sU_pad, nullptr, st);
+int launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
+                  void* sU_pad, float* part, cudaStream_t st) {
+  if (RP == 64) launch_skinny<64, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, st);
+  else launch_skinny<128, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, st);
+  return skinny_splits(M, N) > 1 ? 2 : 1;
 }
 
 // ===========================================================================

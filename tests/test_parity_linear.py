@@ -196,3 +196,43 @@ def test_backward_4096_full_size(q):
     Wd = _oracle_weight(wq, W)
     dXr, _, _ = oracle.linear_bwd(Xn[rows], dYn[rows], Wd, An, Bn, wl.alpha, wl.r)
     assert rel_err(dX[rows], dXr) <= TOL
+
+
+# ---------------------------------------------------------------------------
+# Decode (M <= 16) at full size
+# ---------------------------------------------------------------------------
+
+def _oracle_weight_rows(W_cpu, rows):
+    """Dequantised rows of a double-quantised weight, all by the oracle: the
+    DQ constants come from every block's absmax, the codes of `rows` only
+    (blocks never straddle rows)."""
+    Wn = W_cpu.float().numpy()
+    a = oracle.block_absmax(Wn)
+    qa, s, mu = oracle.double_quantize(a)
+    ah = oracle.dq_absmax(qa, s, mu)
+    nbr = Wn.shape[1] // 64
+    out = []
+    for r in rows:
+        codes, _ = oracle.quantize(Wn[r:r + 1])
+        out.append(oracle.dequantize(oracle.pack(codes), ah[r * nbr:(r + 1) * nbr], (1, Wn.shape[1])))
+    return np.concatenate(out, axis=0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("outliers", [False, True])
+def test_decode_70b_full_size(q, outliers):
+    wl = synth.WORKLOADS["decode_70b"]
+    W = synth.weight(28672, 8192, wl.seed(synth.TID_W), "bf16", outliers=outliers)
+    wq = q.quantize(W.cuda(), double_quant=True)
+    rng = np.random.default_rng(5 + int(outliers))
+    rows = np.unique(np.concatenate([rng.choice(28672, 96, replace=False), [0, 28671]]))
+    Wd = _oracle_weight_rows(W, rows)
+    A = synth.activations(wl.r, 8192, wl.seed(synth.TID_A), sigma=0.02)
+    B = synth.activations(28672, wl.r, wl.seed(synth.TID_B), sigma=0.02)
+    for M in wl.decode_M:
+        X = synth.activations(M, 8192, wl.seed(synth.TID_X) + M)
+        Y, _ = q.linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), wl.alpha)
+        assert q.qlora_check_status() == 0
+        Yr, _ = oracle.linear_fwd(X.float().numpy(), Wd, A.float().numpy(),
+                                  B.float().numpy()[rows], wl.alpha, wl.r)
+        assert rel_err(Y[:, rows], Yr) <= TOL
