@@ -29,11 +29,12 @@ void count_launches(int n);
 struct Nf4Tables {
   float q[16];
   float t[15];
-  // 32 buckets of width 1/16 over [-1, 1): bucket b covers
-  // [-1 + b/16, -1 + (b+1)/16).  At most one threshold falls in a bucket.
-  // code(x) = bucket_base[b] + (x >= bucket_thr[b]).
-  uint8_t bucket_base[32];
-  float bucket_thr[32];
+  // Buckets of width 1/16 around the points -1 + b/16: bucket b covers
+  // [-1 + (b - 0.5)/16, -1 + (b + 0.5)/16), b = 0..32 (index round(16 x + 16)
+  // for x in [-1, 1]); entries 33..63 are unused padding.  At most one
+  // threshold falls in a bucket; code(x) = bucket_base[b] + (x >= bucket_thr[b]).
+  uint8_t bucket_base[64];
+  float bucket_thr[64];
 };
 
 const Nf4Tables& host_tables();   // computed once on the host (table.cpp)

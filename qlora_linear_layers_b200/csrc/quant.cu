@@ -16,100 +16,140 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise: one thread owns 32 consecutive weights, an adjacent lane pair owns
-// one 64-weight block.  absmax is an integer max over |w| bit patterns (exact,
-// and any NaN/Inf shows up as >= 0x7f800000); one shuffle joins the pair.
+// Quantise: one thread owns 8 consecutive weights (one 16-byte bf16 load, a
+// 4-byte code store), 8 adjacent lanes own one 64-weight block, so every warp
+// access is contiguous.  absmax is an integer max over |w| bit patterns
+// (exact; NaN/Inf show up as >= 0x7f800000), joined by 3 shuffles.
+//
+// Code of x = RN32(w / a):  x' = RN32(w * RN32(1/a)) is within 2.5 ulp of x.
+// A 64-entry bucket table over [-1, 1] (width 1/16, index = round(16 x + 16),
+// read with one 8-byte shared load) holds the single threshold T that can
+// fall in the bucket and the number of thresholds below it.  When x' is more
+// than 8 ulp from T, x and x' are on the same side of every threshold and the
+// code is base + (x' >= T); otherwise -- and for blocks whose absmax is 0 or
+// below 2^-125 -- x is computed exactly with the IEEE division (a rarely
+// taken branch, kept out of the unrolled loop).  Thresholds sit >= 1e-4 from bucket edges (checked on the
+// host), so x' may pick the neighbouring bucket near an edge without effect.
 // ===========================================================================
 
-template <typename T> struct Loader;
-
-template <> struct Loader<__nv_bfloat16> {
-  // 32 bf16 = 4 x 16 bytes; returns the fp32 bit patterns.
-  __device__ __forceinline__ static void load(const void* base, int64_t chunk, uint32_t (&u)[32]) {
-    const uint4* p = reinterpret_cast<const uint4*>(base) + chunk * 4;
+// Loaders return the 8 weights as fp32 bit patterns and the max of their
+// magnitudes' bit patterns (bf16: a 16-bit SIMD max over packed pairs).
+template <typename T> struct Loader8;
+template <> struct Loader8<__nv_bfloat16> {
+  __device__ __forceinline__ static uint32_t load(const void* base, int64_t chunk, uint32_t (&u)[8]) {
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(base) + chunk);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t mp = __vmaxu2(__vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
+                           __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint4 q = __ldcs(p + v);
-      uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    for (int j = 0; j < 4; ++j) { u[2 * j] = w[j] << 16; u[2 * j + 1] = w[j] & 0xFFFF0000u; }
+    return max(mp << 16, mp & 0xFFFF0000u);
+  }
+};
+template <> struct Loader8<float> {
+  __device__ __forceinline__ static uint32_t load(const void* base, int64_t chunk, uint32_t (&u)[8]) {
+    const uint4* p = reinterpret_cast<const uint4*>(base) + 2 * chunk;
+    const uint4 a = __ldcs(p), b = __ldcs(p + 1);
+    u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w; u[4] = b.x; u[5] = b.y; u[6] = b.z; u[7] = b.w;
+    uint32_t m = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        u[8 * v + 2 * j] = w[j] << 16;
-        u[8 * v + 2 * j + 1] = w[j] & 0xFFFF0000u;
-      }
-    }
+    for (int i = 0; i < 8; ++i) m = max(m, u[i] & 0x7FFFFFFFu);
+    return m;
   }
 };
 
-template <> struct Loader<float> {
-  __device__ __forceinline__ static void load(const void* base, int64_t chunk, uint32_t (&u)[32]) {
-    const uint4* p = reinterpret_cast<const uint4*>(base) + chunk * 8;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      uint4 q = __ldcs(p + v);
-      u[4 * v] = q.x; u[4 * v + 1] = q.y; u[4 * v + 2] = q.z; u[4 * v + 3] = q.w;
-    }
+struct Bucket { float thr; uint32_t base; };
+
+__device__ __forceinline__ uint32_t bucket_index(float x) {
+  // round(16 x + 16) lands in the low mantissa bits of 16 x + 16 + 2^23
+  return __float_as_uint(fmaf(x, 16.0f, 8388624.0f)) & 63u;
+}
+
+// Exact codes x = RN32(w / a) for the elements of `chunk` flagged in `mask`
+// (rare: a fast quotient within 8 ulp of a threshold, or a zero / tiny absmax
+// block).  The flagged weights are re-read (cached) rather than passed in, so
+// the hot loop keeps its values in registers.
+template <typename T>
+__device__ __noinline__ uint32_t exact_codes(const void* W, int64_t chunk, float a, bool zero_block,
+                                             uint32_t mask, uint32_t out, const Bucket* bks) {
+  for (int i = 0; i < 8; ++i) {
+    if (!((mask >> i) & 1u)) continue;
+    float w;
+    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[chunk * 8 + i]);
+    else w = reinterpret_cast<const float*>(W)[chunk * 8 + i];
+    const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
+    const Bucket bk = bks[bucket_index(x)];
+    const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
+    const int sh = 8 * (i >> 1) + ((i & 1) ? 0 : 4);
+    out = (out & ~(0xFu << sh)) | (code << sh);
   }
-};
+  return out;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256)
 k_nf4_quantize(const void* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ packed,
                float* __restrict__ absmax, Nf4Tables tb, int* status) {
-  __shared__ uint32_t s_base[32];
-  __shared__ float s_thr[32];
-  if (threadIdx.x < 32) {
-    s_base[threadIdx.x] = tb.bucket_base[threadIdx.x];
-    s_thr[threadIdx.x] = tb.bucket_thr[threadIdx.x];
+  __shared__ Bucket s_bk[64];
+  if (threadIdx.x < 64) {
+    const int b = threadIdx.x;
+    s_bk[b].thr = tb.bucket_thr[b];
+    s_bk[b].base = tb.bucket_base[b];
   }
   __syncthreads();
-
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   bool bad = false;
-
-  for (int64_t base = warp * 32; base < nchunks; base += nwarps * 32) {
-    const int64_t chunk = base + lane;
-    const bool active = chunk < nchunks;      // uniform over each lane pair (nchunks even)
-    uint32_t u[32];
-    uint32_t m = 0;
-    if (active) {
-      Loader<T>::load(W, chunk, u);
+  // Two chunks per iteration (both loads in flight before either is used);
+  // every lane of a warp runs the same number of iterations (shuffles below).
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nchunks;
+       base += 2 * stride) {
+    uint32_t u[2][8], mloc[2] = {0u, 0u};
+    int64_t chunk[2];
+    bool active[2];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) m = max(m, u[i] & 0x7FFFFFFFu);
+    for (int h = 0; h < 2; ++h) {
+      chunk[h] = base + h * stride + lane;
+      active[h] = chunk[h] < nchunks;             // whole 8-lane groups (nchunks % 8 == 0)
+      if (active[h]) mloc[h] = Loader8<T>::load(W, chunk[h], u[h]);
     }
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    if (!active) continue;
-    if (m >= 0x7F800000u) { bad = true; m = 0; }
-    const float a = __uint_as_float(m);
-
-    uint32_t out[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      // x = RN32(w / a); an all-zero block has x = 0 everywhere.
-      const float w = __uint_as_float(u[i]);
-      const float x = (m == 0) ? 0.0f : __fdiv_rn(w, a);
-      int b = __float2int_rz(__fmul_rn(__fadd_rn(x, 1.0f), 16.0f));
-      b = min(max(b, 0), 31);
-      const uint32_t code = s_base[b] + (x >= s_thr[b] ? 1u : 0u);
-      // byte j of the 16-byte output holds elements 2j (high) and 2j+1 (low);
-      // little-endian: byte j sits at bits 8*(j%4) of word j/4.
-      const int byte = i >> 1;
-      const int shift = 8 * (byte & 3) + ((i & 1) ? 0 : 4);
-      out[byte >> 2] |= code << shift;
+    for (int h = 0; h < 2; ++h) {
+      uint32_t m = mloc[h];
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      if (!active[h]) continue;
+      if (m >= 0x7F800000u) { bad = true; m = 0; }
+      const float a = __uint_as_float(m);
+      const bool exact_block = m < 0x01000000u;   // a == 0 or a < 2^-125
+      const float inv = exact_block ? 0.0f : __frcp_rn(a);
+      uint32_t out = 0;
+      bool anynear = exact_block;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float x = __fmul_rn(__uint_as_float(u[h][i]), inv);
+        const Bucket bk = s_bk[bucket_index(x)];
+        // within 8 ulp of the threshold (same sign there, so the bit patterns
+        // differ by the ulp distance): decide exactly below
+        anynear |= (uint32_t)(__float_as_int(x) - __float_as_int(bk.thr) + 8) <= 16u;
+        const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
+        // element 2j -> high nibble of byte j; byte j at bits 8j (fields disjoint: add = or)
+        out += code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+      }
+      if (anynear) out = exact_codes<T>(W, chunk[h], a, m == 0, 0xFFu, out, s_bk);
+      reinterpret_cast<uint32_t*>(packed)[chunk[h]] = out;
+      if ((lane & 7) == 0) absmax[chunk[h] >> 3] = a;
     }
-    reinterpret_cast<uint4*>(packed)[chunk] = make_uint4(out[0], out[1], out[2], out[3]);
-    if ((lane & 1) == 0) absmax[chunk >> 1] = a;
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
 }
 
 void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
                      int* status, cudaStream_t s, int num_sms) {
-  const int64_t nchunks = n / 32;
+  const int64_t nchunks = n / 8;
   const int threads = 256;
-  int64_t want = (nchunks + threads - 1) / threads;
-  int blocks = (int)std::min<int64_t>(want, (int64_t)num_sms * 8);
+  int blocks = (int)std::min<int64_t>((nchunks + threads - 1) / threads, (int64_t)num_sms * 8);
   blocks = std::max(blocks, 1);
   const Nf4Tables& tb = host_tables();
   if (dtype == QLORA_BF16)
@@ -168,8 +208,12 @@ k_absmax_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* _
 // 2^-149 (the value of a float with exponent field e and significand m is
 // m * 2^(max(e,1) - 150)); round S to the nearest double (ties to even), then
 // mean = RN32(RN64(S * 2^-149) / n).
-__global__ void k_mean_finalize(const unsigned long long* __restrict__ hist, int64_t n,
-                                float* __restrict__ mean) {
+__global__ void __launch_bounds__(256)
+k_mean_finalize(const unsigned long long* __restrict__ hist_g, int64_t n,
+                float* __restrict__ mean) {
+  __shared__ unsigned long long hist[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = hist_g[i];   // parallel loads
+  __syncthreads();
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   constexpr int L = 12;                  // 384-bit accumulator
   uint32_t acc[L];
@@ -258,14 +302,15 @@ void launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, flo
   cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
   int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 4);
   k_absmax_hist<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, hist, status);
-  k_mean_finalize<<<1, 32, 0, s>>>(hist, n, dq_mean);
+  k_mean_finalize<<<1, 256, 0, s>>>(hist, n, dq_mean);
   const int64_t ngroups = (n + 255) / 256;
   blocks = (int)std::min<int64_t>((ngroups + 7) / 8, (int64_t)num_sms * 8);
   k_dq_blockwise<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, dq_mean, qabsmax, dq_scale);
 }
 
 // ===========================================================================
-// Dequantise: one thread owns 32 weights (16 packed bytes -> 64 output bytes).
+// Dequantise: one thread owns 8 weights (a 4-byte code load, a 16-byte bf16
+// store; contiguous per warp), 8 lanes share a block's scale.
 // w' = RNbf16(RN32(q[code] * a^)), a^ recovered from the double-quantised
 // constants as RN32(RN32(RN32(c / 127) * s_g) + mean).
 // ===========================================================================
@@ -277,40 +322,32 @@ k_nf4_dequantize(const uint8_t* __restrict__ packed, int64_t nchunks,
                  const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
                  uint4* __restrict__ out, Nf4Tables tb) {
   __shared__ float s_q[16];
+  __shared__ float s_inv127[256];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
+  s_inv127[threadIdx.x] = __fdiv_rn((float)((int)threadIdx.x - 127), 127.0f);
   __syncthreads();
   const float mu = DQ ? dq_mean[0] : 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < nchunks;
        chunk += stride) {
-    const int64_t blk = chunk >> 1;
+    const int64_t blk = chunk >> 3;
     float a;
-    if (DQ) {
-      const float c = (float)qabsmax[blk];
-      a = __fadd_rn(__fmul_rn(__fdiv_rn(c, 127.0f), dq_scale[blk >> 8]), mu);
-    } else {
-      a = absmax[blk];
-    }
-    const uint4 pk = __ldcs(reinterpret_cast<const uint4*>(packed) + chunk);
-    const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
-    uint32_t o[16];
+    if (DQ) a = __fadd_rn(__fmul_rn(s_inv127[qabsmax[blk] + 127], __ldg(dq_scale + (blk >> 8))), mu);
+    else a = __ldg(absmax + blk);
+    const uint32_t wd = __ldcs(reinterpret_cast<const uint32_t*>(packed) + chunk);
+    uint32_t o[4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {            // byte j -> elements 2j (hi), 2j+1 (lo)
-      const uint32_t byte = (wds[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-      const float v0 = __fmul_rn(s_q[byte >> 4], a);
-      const float v1 = __fmul_rn(s_q[byte & 15], a);
-      o[j] = pack_bf16x2(v0, v1);
+    for (int j = 0; j < 4; ++j) {            // byte j -> elements 2j (high nibble), 2j+1 (low)
+      const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
+      o[j] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], a), __fmul_rn(s_q[byte & 15], a));
     }
-    uint4* dst = out + chunk * 4;
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-      __stcs(dst + v, make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]));
+    __stcs(out + chunk, make_uint4(o[0], o[1], o[2], o[3]));
   }
 }
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms) {
   const int64_t n = w->rows * w->cols;
-  const int64_t nchunks = n / 32;
+  const int64_t nchunks = n / 8;
   int blocks = (int)std::min<int64_t>((nchunks + 255) / 256, (int64_t)num_sms * 8);
   blocks = std::max(blocks, 1);
   const Nf4Tables& tb = host_tables();

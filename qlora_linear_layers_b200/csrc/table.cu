@@ -68,14 +68,14 @@ static Nf4Tables build_tables() {
   // must sit well away from a bucket edge so that the rounding in the
   // bucket index (x + 1) * 16 can never put x on the wrong side of an edge
   // that a threshold shares.
-  for (int b = 0; b < 32; ++b) {
-    double lo = -1.0 + b / 16.0, hi = lo + 1.0 / 16.0;
+  for (int b = 0; b < 64; ++b) {
+    double lo = -1.0 + (b - 0.5) / 16.0, hi = lo + 1.0 / 16.0;
     int base = 0;
-    float thr = INFINITY;
+    float thr = 2.0f;                         // "no threshold here": above every |x| <= 1
     for (int j = 0; j < 15; ++j) {
       if ((double)tb.t[j] < lo) ++base;
       else if ((double)tb.t[j] < hi) {
-        if (thr != INFINITY) { std::fprintf(stderr, "qlora_nf4: two thresholds in a bucket\n"); std::abort(); }
+        if (thr != 2.0f) { std::fprintf(stderr, "qlora_nf4: two thresholds in a bucket\n"); std::abort(); }
         thr = tb.t[j];
       }
       double edge_gap = std::min(std::fabs((double)tb.t[j] - lo), std::fabs((double)tb.t[j] - hi));
