@@ -319,7 +319,9 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);
-  st = launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
+  // paired-SM tiles (256 weight rows) once there is more than one 128-row block
+  st = N > 128 ? launch_qlora_gemm_pair(a, X, sT, RP, s, d->sms)
+               : launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;
   st = launch_status();

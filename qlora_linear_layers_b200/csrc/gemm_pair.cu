@@ -1,0 +1,334 @@
+// Fused NF4-dequant QLoRA forward GEMM on paired SMs (tcgen05 cta_group::2).
+//
+//   Y = X deq(W)^T + (s T) B^T
+//
+// Same computation and layout rules as the single-CTA engine in gemm.cu (page
+// "QLoRA Explained", section "Why the expansion cannot be skipped": codes ->
+// table -> block scale -> bf16 -> tensor core), with two SMs of a cluster
+// sharing each 256 x 256 output tile:
+//  * MMA M = 256 (CTA r owns weight rows 128r..128r+127 of the tile, written
+//    by its own converter warps into its own TMEM), MMA N = 256 (CTA r loads
+//    tokens 128r..128r+127 of the tile into its own shared memory).  Each SM
+//    thus streams half the token tile per K step that a single-CTA 128 x 256
+//    tile needs, halving the shared-memory port traffic (TMA writes + MMA
+//    reads of the token operand), which is what bounds the single-CTA kernel.
+//  * The even CTA's elected thread issues tcgen05.mma.cta_group::2 and
+//    commits with an arrival multicast to both CTAs' "empty" and "full"
+//    barriers.  Both CTAs' TMA loads (no multicast: each CTA loads its own
+//    half) complete on the even CTA's "full" barrier; the odd CTA's converter
+//    and epilogue warps arrive on the even CTA's barriers through mapa.
+//  * 8 pipeline stages: 16 KB of tokens per CTA per stage, A ring of 8 x 32
+//    TMEM columns beside the 256-column accumulator (all 512 columns).
+// Every wait is bounded (status QLORA_ERR_TIMEOUT); both CTAs meet at a
+// cluster barrier before the paired TMEM is released.
+
+#include <algorithm>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "gemm.h"
+#include "nf4_lut.cuh"
+
+namespace qnf4 {
+
+namespace pair {
+
+constexpr int BN = 128;          // weight rows per CTA (MMA M = 256 per pair)
+constexpr int BM = 256;          // tokens per pair tile (MMA N)
+constexpr int BMH = BM / 2;      // tokens loaded by each CTA
+constexpr int BK = 64;           // contraction per stage (= one NF4 block)
+constexpr int NS = 8;            // pipeline stages
+constexpr int X_BYTES = BMH * BK * 2;            // 16 KB per CTA per stage
+constexpr int ACC_COL = 0;                       // accumulator: TMEM columns [0, 256)
+constexpr int A_COL = 256;                       // A ring: NS x 32 columns
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 448;                 // 14 warps
+constexpr int EPI_WARP0 = 2;                     // warps 2-5: epilogue
+constexpr int CVT_WARP0 = 6;                     // warps 6-13: A-operand producers
+constexpr uint16_t kBoth = 0x3;                  // cluster CTA mask of the pair
+
+struct Smem {
+  uint8_t x[NS][X_BYTES];
+  uint64_t x_full[NS], x_empty[NS];
+  uint64_t a_full[NS], a_empty[NS];
+  uint64_t acc_full, acc_empty, done;
+  uint32_t tmem_base;
+  int abort;
+  float inv127[256];
+};
+
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+
+template <bool DQ>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
+                  const __grid_constant__ CUtensorMap tm_tokad,   // [Mtok, RP]  bf16
+                  const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();        // 0: issues the MMAs
+  const bool leader = rank == 0;
+
+  const int n_pairs_n = (p.Nout + 2 * BN - 1) / (2 * BN);
+  const int n_tiles = n_pairs_n * ((p.Mtok + BM - 1) / BM);
+  const int cluster = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
+  const int nk = p.Kc / BK;
+  const int nsteps = nk + p.na;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&S.x_full[i], 1);                  // leader's expect_tx; tx from both CTAs
+      mbar_init(&S.x_empty[i], 1);                 // multicast commit
+      mbar_init(&S.a_full[i], 8);                  // 4 converter warps per CTA
+      mbar_init(&S.a_empty[i], 1);                 // multicast commit
+    }
+    mbar_init(&S.acc_full, 1);                     // multicast commit
+    mbar_init(&S.acc_empty, 8);                    // 4 epilogue warps per CTA
+    mbar_init(&S.done, 1);
+    S.abort = 0;
+    mbar_fence_init();
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    S.inv127[i] = __fdiv_rn((float)(i - 127), 127.0f);
+  if (warp == 1) {
+    tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_tok);
+    tma_prefetch_desc(&tm_tokad);
+  }
+  tc_fence_before();
+  cluster_sync();                                  // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  volatile int* abort = &S.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t xi = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < n_tiles && ok; tile += n_clusters) {
+        const int m0 = (tile / n_pairs_n) * BM + (int)rank * BMH;
+        for (int ks = 0; ks < nsteps; ++ks, ++xi) {
+          const int s = xi % NS;
+          if (!(ok = mbar_wait_cluster(&S.x_empty[s], ((xi / NS) & 1) ^ 1, abort, p.status))) break;
+          if (leader) mbar_arrive_expect_tx(&S.x_full[s], 2 * X_BYTES);
+          const bool ad = ks >= nk;
+          const uint32_t full0 = mapa_shared(smem_u32(&S.x_full[s]), 0);
+          tma_load_2d_pair(S.x[s], ad ? &tm_tokad : &tm_tok, full0, (ad ? ks - nk : ks) * BK, m0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BN, BM);
+      uint32_t xi = 0, lt = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < n_tiles && ok; tile += n_clusters, ++lt) {
+        ok = mbar_wait_cluster(&S.acc_empty, (lt & 1) ^ 1, abort, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nsteps && ok; ++ks, ++xi) {
+          const int s = xi % NS;
+          const uint32_t par = (xi / NS) & 1;
+          ok = mbar_wait_cluster(&S.x_full[s], par, abort, p.status) &&
+               mbar_wait_cluster(&S.a_full[s], par, abort, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ts_pair(tmem + ACC_COL, tmem + A_COL + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
+                        idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_pair_mc(&S.x_empty[s], kBoth);
+          mma_commit_pair_mc(&S.a_empty[s], kBoth);
+        }
+        if (ok) mma_commit_pair_mc(&S.acc_full, kBoth);
+      }
+      // all MMAs issued by this thread are complete once `done` flips
+      mma_commit_pair_mc(&S.done, 0x1);
+      mbar_wait(&S.done, 0, abort, p.status);
+    }
+  } else if (warp >= CVT_WARP0) {
+    // ------------------------------------------------------------ A-operand producers (TMEM)
+    // Step ks < nk: NF4 -> bf16 for block ks of the thread's weight row; step
+    // ks >= nk: 64 bf16 of the row's adapter factor B (zero-padded to RP).
+    const int quad = warp & 3;
+    const uint32_t par = (uint32_t)((warp - CVT_WARP0) >> 2);   // steps of this parity
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
+    const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
+    const int64_t kb_per_row = p.Kc / 64;
+    struct Src { uint4 c[8]; float a_raw, sg; int qa; bool valid, ad; };
+    auto fetch = [&](uint32_t ai, Src& d) -> bool {
+      const uint32_t lt = ai / (uint32_t)nsteps;
+      const int ks = (int)(ai - lt * (uint32_t)nsteps);
+      const int tile = cluster + (int)lt * n_clusters;
+      if (tile >= n_tiles) return false;
+      const int n = (tile % n_pairs_n) * (2 * BN) + (int)rank * BN + row_in_tile;
+      d.valid = n < p.Nout;
+      d.ad = ks >= nk;
+      const int64_t nn = d.valid ? n : 0;
+      if (d.ad) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.wad + nn * p.RP + (ks - nk) * BK);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d.c[i] = __ldcg(src + i);
+      } else {
+        const uint4* codes = reinterpret_cast<const uint4*>(p.packed + nn * (p.Kc / 2)) + 2 * ks;
+        d.c[0] = __ldcg(codes);
+        d.c[1] = __ldcg(codes + 1);
+        const int64_t b = nn * kb_per_row + ks;
+        if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); d.a_raw = 0.f; }
+        else { d.a_raw = __ldcg(p.absmax + b); d.qa = 0; d.sg = 0.f; }
+      }
+      return true;
+    };
+    Src cur, nxt;
+    uint32_t ai = par;
+    bool have = fetch(ai, cur);
+    while (have) {
+      const bool more = fetch(ai + 2, nxt);       // prefetch this warp's next step
+      uint32_t v[32];
+      if (!cur.valid) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      } else if (cur.ad) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[4 * i] = cur.c[i].x; v[4 * i + 1] = cur.c[i].y;
+          v[4 * i + 2] = cur.c[i].z; v[4 * i + 3] = cur.c[i].w;
+        }
+      } else {
+        // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
+        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 127], cur.sg), mu) : cur.a_raw;
+        const Lut l = build_lut(a, p.q);
+        const uint32_t wds[8] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w,
+                                 cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
+      }
+      const int sa = ai % NS;
+      if (!mbar_wait_cluster(&S.a_empty[sa], ((ai / NS) & 1) ^ 1, abort, p.status)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem + tmem_lane + A_COL + sa * 32;
+      tmem_st16(taddr, v);
+      tmem_st16(taddr + 16, v + 16);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.a_full[sa]), 0));
+      cur = nxt;
+      have = more;
+      ai += 2;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
+    constexpr int HALF = BM / 2;                 // columns drained per round
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
+    const bool odd = lane & 1;
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(&S.acc_empty), 0);
+    uint32_t lt = 0;
+    for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++lt) {
+      const int n0 = (tile % n_pairs_n) * (2 * BN) + (int)rank * BN;
+      const int mt = (tile / n_pairs_n) * BM;
+      if (!mbar_wait_cluster(&S.acc_full, lt & 1, abort, p.status)) break;
+      __syncwarp();
+      tc_fence_after();
+      // lane pairs (o, o+1) swap halves so each lane stores two adjacent
+      // outputs of one token row: even lanes row m, odd lanes row m+1
+      const int ocol = n0 + row_in_tile - (odd ? 1 : 0);
+      const int step = p.Nout;                   // two bf16 rows = Nout words
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t packed[HALF / 2];
+#pragma unroll
+        for (int c = 0; c < HALF; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + tmem_lane + ACC_COL + h * HALF + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            packed[c / 2 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        }
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc_empty0);
+        }
+        const int mfirst = mt + h * HALF + (odd ? 1 : 0);
+        const int rows_left = (ocol < p.Nout) ? p.Mtok - mfirst : 0;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (int64_t)mfirst * p.Nout + ocol);
+#pragma unroll
+        for (int c = 0; c < HALF; c += 2) {
+          const uint32_t mine = packed[c / 2];
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          const uint32_t out = odd ? prmt(other, mine, 0x7632) : prmt(mine, other, 0x5410);
+          if (c < rows_left) *dst = out;
+          dst += step;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();                                  // both CTAs done with the paired TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace pair
+
+// Paired-SM forward GEMM (MODE_NF4 only).  Returns QLORA_OK or QLORA_ERR_CUDA.
+int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad, int RP,
+                           cudaStream_t s, int num_sms) {
+  using namespace pair;
+  CUtensorMap t_tok, t_tokad;
+  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, BMH)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, BMH)) return QLORA_ERR_CUDA;
+  const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + BM - 1) / BM);
+  const int clusters = std::max(1, std::min(n_tiles, num_sms / 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static bool attr_set[2] = {false, false};
+  cudaError_t e;
+  if (a.double_quant) {
+    if (!attr_set[1]) {
+      cudaFuncSetAttribute(k_qlora_gemm_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      attr_set[1] = true;
+    }
+    e = cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<true>, t_tok, t_tokad, a);
+  } else {
+    if (!attr_set[0]) {
+      cudaFuncSetAttribute(k_qlora_gemm_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      attr_set[0] = true;
+    }
+    e = cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<false>, t_tok, t_tokad, a);
+  }
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+}  // namespace qnf4
