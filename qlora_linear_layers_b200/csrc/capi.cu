@@ -320,7 +320,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);
   // paired-SM tiles (256 weight rows) once there is more than one 128-row block
-  st = N > 128 ? launch_qlora_gemm_pair(a, X, sT, RP, s, d->sms)
+  st = N > 128 ? launch_qlora_gemm_pair(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms)
                : launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;
@@ -375,7 +375,8 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);
-  st = launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
+  st = K > 128 ? launch_qlora_gemm_pair(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms)
+               : launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;
   // dA[r, K] = (s U)^T X ;  dB[N, r] = s dY^T T

@@ -31,10 +31,11 @@ struct GemmArgs {
   float q[16];                // NF4 table
 };
 
-// Paired-SM (cluster of 2, tcgen05 cta_group::2) form of the MODE_NF4 GEMM:
-// 256 x 256 output tiles; tok: [Mtok, Kc]; tokad: [Mtok, RP]; weights from `a`.
-int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad, int RP,
-                           cudaStream_t s, int num_sms);
+// Paired-SM (cluster of 2, tcgen05 cta_group::2) form of the GEMM: 256 x 256
+// output tiles; tok: [Mtok, Kc]; tokad: [Mtok, RP]; MODE_NF4 weights from
+// `a`, MODE_BF16 weights w [Nout, Kc] and wad [Nout, RP].
+int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
+                           const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);
 
 // tok: [Mtok, Kc]; tokad: [Mtok, RP]; wad: [Nout, RP]; w: [Nout, Kc] (MODE_BF16 only).
 int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* tokad,

@@ -1,6 +1,7 @@
-// Fused NF4-dequant QLoRA forward GEMM on paired SMs (tcgen05 cta_group::2).
+// QLoRA GEMMs on paired SMs (tcgen05 cta_group::2).
 //
-//   Y = X deq(W)^T + (s T) B^T
+//   MODE_NF4  (forward):      Y  = X deq(W)^T + (s T) B^T
+//   MODE_BF16 (backward dX):  dX = dY deq(W) + (s U) A     (weights as deq(W)^T, bf16)
 //
 // Same computation and layout rules as the single-CTA engine in gemm.cu (page
 // "QLoRA Explained", section "Why the expansion cannot be skipped": codes ->
@@ -17,8 +18,10 @@
 //    barriers.  Both CTAs' TMA loads (no multicast: each CTA loads its own
 //    half) complete on the even CTA's "full" barrier; the odd CTA's converter
 //    and epilogue warps arrive on the even CTA's barriers through mapa.
-//  * 8 pipeline stages: 16 KB of tokens per CTA per stage, A ring of 8 x 32
+//  * MODE_NF4: 8 pipeline stages of 16 KB of tokens per CTA, A ring of 8 x 32
 //    TMEM columns beside the 256-column accumulator (all 512 columns).
+//  * MODE_BF16: both operands by TMA (each CTA its 128 weight rows and its
+//    128 tokens), 6 stages of 16 + 16 KB; the converter warps stay idle.
 // Every wait is bounded (status QLORA_ERR_TIMEOUT); both CTAs meet at a
 // cluster barrier before the paired TMEM is released.
 
@@ -40,18 +43,23 @@ constexpr int BN = 128;          // weight rows per CTA (MMA M = 256 per pair)
 constexpr int BM = 256;          // tokens per pair tile (MMA N)
 constexpr int BMH = BM / 2;      // tokens loaded by each CTA
 constexpr int BK = 64;           // contraction per stage (= one NF4 block)
-constexpr int NS = 8;            // pipeline stages
+template <int MODE> __host__ __device__ constexpr int stages() { return MODE == MODE_NF4 ? 8 : 6; }
 constexpr int X_BYTES = BMH * BK * 2;            // 16 KB per CTA per stage
 constexpr int ACC_COL = 0;                       // accumulator: TMEM columns [0, 256)
-constexpr int A_COL = 256;                       // A ring: NS x 32 columns
+constexpr int A_COL = 256;                       // MODE_NF4 A ring: 8 x 32 columns
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 448;                 // 14 warps
 constexpr int EPI_WARP0 = 2;                     // warps 2-5: epilogue
 constexpr int CVT_WARP0 = 6;                     // warps 6-13: A-operand producers
 constexpr uint16_t kBoth = 0x3;                  // cluster CTA mask of the pair
 
+constexpr int W_BYTES = BN * BK * 2;             // 16 KB weight tile per CTA (MODE_BF16)
+
+template <int MODE>
 struct Smem {
+  static constexpr int NS = stages<MODE>();
   uint8_t x[NS][X_BYTES];
+  uint8_t w[MODE == MODE_BF16 ? NS : 1][MODE == MODE_BF16 ? W_BYTES : 16];
   uint64_t x_full[NS], x_empty[NS];
   uint64_t a_full[NS], a_empty[NS];
   uint64_t acc_full, acc_empty, done;
@@ -60,15 +68,20 @@ struct Smem {
   float inv127[256];
 };
 
-constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+template <int MODE>
+constexpr size_t smem_bytes() { return sizeof(Smem<MODE>) + 1024; }
 
-template <bool DQ>
+template <int MODE, bool DQ>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
                   const __grid_constant__ CUtensorMap tm_tokad,   // [Mtok, RP]  bf16
+                  const __grid_constant__ CUtensorMap tm_w,       // [Nout, Kc]  bf16 (MODE_BF16)
+                  const __grid_constant__ CUtensorMap tm_wad,     // [Nout, RP]  bf16 (MODE_BF16)
                   const GemmArgs p) {
+  constexpr int NS = stages<MODE>();
   extern __shared__ uint8_t smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<MODE>& S =
+      *reinterpret_cast<Smem<MODE>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();        // 0: issues the MMAs
@@ -78,7 +91,7 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   const int n_tiles = n_pairs_n * ((p.Mtok + BM - 1) / BM);
   const int cluster = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
-  const int nk = p.Kc / BK;
+  const int nk = (p.Kc + BK - 1) / BK;
   const int nsteps = nk + p.na;
 
   if (threadIdx.x == 0) {
@@ -103,6 +116,10 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_tok);
     tma_prefetch_desc(&tm_tokad);
+    if (MODE == MODE_BF16) {
+      tma_prefetch_desc(&tm_w);
+      tma_prefetch_desc(&tm_wad);
+    }
   }
   tc_fence_before();
   cluster_sync();                                  // barriers of both CTAs initialised
@@ -117,13 +134,16 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
       bool ok = true;
       for (int tile = cluster; tile < n_tiles && ok; tile += n_clusters) {
         const int m0 = (tile / n_pairs_n) * BM + (int)rank * BMH;
+        const int n0 = (tile % n_pairs_n) * (2 * BN) + (int)rank * BN;
         for (int ks = 0; ks < nsteps; ++ks, ++xi) {
           const int s = xi % NS;
           if (!(ok = mbar_wait_cluster(&S.x_empty[s], ((xi / NS) & 1) ^ 1, abort, p.status))) break;
-          if (leader) mbar_arrive_expect_tx(&S.x_full[s], 2 * X_BYTES);
+          if (leader) mbar_arrive_expect_tx(&S.x_full[s], 2 * (X_BYTES + (MODE == MODE_BF16 ? W_BYTES : 0)));
           const bool ad = ks >= nk;
+          const int kc = (ad ? ks - nk : ks) * BK;
           const uint32_t full0 = mapa_shared(smem_u32(&S.x_full[s]), 0);
-          tma_load_2d_pair(S.x[s], ad ? &tm_tokad : &tm_tok, full0, (ad ? ks - nk : ks) * BK, m0);
+          tma_load_2d_pair(S.x[s], ad ? &tm_tokad : &tm_tok, full0, kc, m0);
+          if (MODE == MODE_BF16) tma_load_2d_pair(S.w[s], ad ? &tm_wad : &tm_w, full0, kc, n0);
         }
       }
     }
@@ -140,17 +160,26 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
         for (int ks = 0; ks < nsteps && ok; ++ks, ++xi) {
           const int s = xi % NS;
           const uint32_t par = (xi / NS) & 1;
-          ok = mbar_wait_cluster(&S.x_full[s], par, abort, p.status) &&
-               mbar_wait_cluster(&S.a_full[s], par, abort, p.status);
+          ok = mbar_wait_cluster(&S.x_full[s], par, abort, p.status);
+          if (ok && MODE == MODE_NF4) ok = mbar_wait_cluster(&S.a_full[s], par, abort, p.status);
           if (!ok) break;
           tc_fence_after();
           const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
+          if (MODE == MODE_NF4) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ts_pair(tmem + ACC_COL, tmem + A_COL + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
-                        idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-          mma_commit_pair_mc(&S.x_empty[s], kBoth);
-          mma_commit_pair_mc(&S.a_empty[s], kBoth);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_ts_pair(tmem + ACC_COL, tmem + A_COL + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
+                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_pair_mc(&S.x_empty[s], kBoth);
+            mma_commit_pair_mc(&S.a_empty[s], kBoth);
+          } else {
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[s]));
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_ss_pair(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_pair_mc(&S.x_empty[s], kBoth);
+          }
         }
         if (ok) mma_commit_pair_mc(&S.acc_full, kBoth);
       }
@@ -160,8 +189,10 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     }
   } else if (warp >= CVT_WARP0) {
     // ------------------------------------------------------------ A-operand producers (TMEM)
-    // Step ks < nk: NF4 -> bf16 for block ks of the thread's weight row; step
-    // ks >= nk: 64 bf16 of the row's adapter factor B (zero-padded to RP).
+    // MODE_NF4 only.  Step ks < nk: NF4 -> bf16 for block ks of the thread's
+    // weight row; step ks >= nk: 64 bf16 of the row's adapter factor B
+    // (zero-padded to RP).
+    if (MODE == MODE_NF4) {
     const int quad = warp & 3;
     const uint32_t par = (uint32_t)((warp - CVT_WARP0) >> 2);   // steps of this parity
     const int row_in_tile = quad * 32 + lane;
@@ -231,6 +262,7 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
       have = more;
       ai += 2;
     }
+    }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
     constexpr int HALF = BM / 2;                 // columns drained per round
@@ -290,21 +322,19 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   }
 }
 
-}  // namespace pair
-
-// Paired-SM forward GEMM (MODE_NF4 only).  Returns QLORA_OK or QLORA_ERR_CUDA.
-int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad, int RP,
-                           cudaStream_t s, int num_sms) {
-  using namespace pair;
-  CUtensorMap t_tok, t_tokad;
-  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, BMH)) return QLORA_ERR_CUDA;
-  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, BMH)) return QLORA_ERR_CUDA;
-  const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + BM - 1) / BM);
-  const int clusters = std::max(1, std::min(n_tiles, num_sms / 2));
+template <int MODE, bool DQ>
+static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
+                               const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(k_qlora_gemm_pair<MODE, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<MODE>());
+    attr_set = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_bytes<MODE>();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -313,21 +343,32 @@ int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  static bool attr_set[2] = {false, false};
-  cudaError_t e;
-  if (a.double_quant) {
-    if (!attr_set[1]) {
-      cudaFuncSetAttribute(k_qlora_gemm_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-      attr_set[1] = true;
-    }
-    e = cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<true>, t_tok, t_tokad, a);
+  return cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<MODE, DQ>, a0, a1, a2, a3, a);
+}
+
+}  // namespace pair
+
+// Paired-SM GEMM.  MODE_NF4: weights from `a` (NF4); MODE_BF16: w [Nout, Kc]
+// and wad [Nout, RP] bf16 by TMA.  Returns QLORA_OK or QLORA_ERR_CUDA.
+int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
+                           const void* wad, const void* w, int RP, cudaStream_t s, int num_sms) {
+  using namespace pair;
+  CUtensorMap t_tok, t_tokad, t_w, t_wad;
+  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, BMH)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, BMH)) return QLORA_ERR_CUDA;
+  if (mode == MODE_BF16) {
+    if (!make_tmap_2d_bf16(&t_w, w, a.Kc, a.Nout, a.Kc, BK, BN)) return QLORA_ERR_CUDA;
+    if (!make_tmap_2d_bf16(&t_wad, wad, RP, a.Nout, RP, BK, BN)) return QLORA_ERR_CUDA;
   } else {
-    if (!attr_set[0]) {
-      cudaFuncSetAttribute(k_qlora_gemm_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-      attr_set[0] = true;
-    }
-    e = cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<false>, t_tok, t_tokad, a);
+    t_w = t_tok;                                   // unused
+    t_wad = t_tokad;
   }
+  const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + BM - 1) / BM);
+  const int clusters = std::max(1, std::min(n_tiles, num_sms / 2));
+  cudaError_t e;
+  if (mode == MODE_BF16) e = launch_pair<MODE_BF16, false>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  else if (a.double_quant) e = launch_pair<MODE_NF4, true>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  else e = launch_pair<MODE_NF4, false>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
