@@ -286,8 +286,9 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   if (M <= kDecodeMaxTokens) {
     // decode-sized call: HBM-bound GEMV on the warp-level tensor cores
     const int n = launch_qlora_gemv(w, X, (int)M, A, B, r, scale, Y, T_save,
-                                    reinterpret_cast<float*>(wsb + lay.gemv), host_tables().q, s,
-                                    d->sms);
+                                    reinterpret_cast<float*>(wsb + lay.gemv), host_tables().q,
+                                    d->status, s, d->sms);
+    if (n < 0) return QLORA_ERR_CUDA;
     st = launch_status();
     if (!st) count_launches(n);
     return st;

@@ -43,16 +43,26 @@ int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* 
 
 // Decode-sized forward (M <= 16): Y = X deq(W)^T + s (X A^T) B^T, T_save =
 // RNbf16(X A^T) when not null.  `part` holds gemv_workspace_bytes(M, N, K, r)
-// bytes.  Returns the number of kernels launched.
+// bytes.  Returns the number of kernels launched, or -1 when the tensor map
+// of the codes cannot be built.  Waits that give up set QLORA_ERR_TIMEOUT in
+// `status`.
 constexpr int kDecodeMaxTokens = 16;
 int launch_qlora_gemv(const nf4_weight* w, const void* X, int M, const void* A, const void* B,
                       int r, float s, void* Y, void* T_save, float* part, const float* q,
-                      cudaStream_t st, int num_sms);
+                      int* status, cudaStream_t st, int num_sms);
 size_t gemv_workspace_bytes(int M, int N, int K, int r);
 
 // 2-D bf16 tensor map, 128-byte swizzle, box [box_outer rows x box_inner cols].
 bool make_tmap_2d_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer);
+// Same for a uint8 matrix: inner extent and row stride in bytes; 128-byte
+// swizzle (box_inner <= 128) or none.
+bool make_tmap_2d_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+// 3-D tiled map (uint8 or bf16): extents (innermost first), strides of
+// dimensions 1 and 2 in bytes (multiples of 16), box extents.
+bool make_tmap_3d(CUtensorMap* tm, const void* base, bool bf16, const uint64_t dims[3],
+                  const uint64_t strides_bytes[2], const uint32_t box[3], bool swizzle128);
 
 // T = X A^T on tensor cores (mma.sync), written as
 //   sT_pad[M, RP] = RNbf16(s * T)  (zero for columns >= r; may be null)

@@ -40,11 +40,10 @@ namespace qnf4 {
 namespace pair {
 
 constexpr int BN = 128;          // weight rows per CTA (MMA M = 256 per pair)
-constexpr int BM = 256;          // tokens per pair tile (MMA N)
-constexpr int BMH = BM / 2;      // tokens loaded by each CTA
 constexpr int BK = 64;           // contraction per stage (= one NF4 block)
 template <int MODE> __host__ __device__ constexpr int stages() { return MODE == MODE_NF4 ? 8 : 6; }
-constexpr int X_BYTES = BMH * BK * 2;            // 16 KB per CTA per stage
+// BM (template argument, a multiple of 32 up to 256): tokens per pair tile =
+// MMA N; each CTA loads BM / 2 tokens, BM * 64 bytes per stage.
 constexpr int ACC_COL = 0;                       // accumulator: TMEM columns [0, 256)
 constexpr int A_COL = 256;                       // MODE_NF4 A ring: 8 x 32 columns
 constexpr int TMEM_COLS = 512;
@@ -55,10 +54,10 @@ constexpr uint16_t kBoth = 0x3;                  // cluster CTA mask of the pair
 
 constexpr int W_BYTES = BN * BK * 2;             // 16 KB weight tile per CTA (MODE_BF16)
 
-template <int MODE>
+template <int MODE, int BM>
 struct Smem {
   static constexpr int NS = stages<MODE>();
-  uint8_t x[NS][X_BYTES];
+  uint8_t x[NS][BM * BK];
   uint8_t w[MODE == MODE_BF16 ? NS : 1][MODE == MODE_BF16 ? W_BYTES : 16];
   uint64_t x_full[NS], x_empty[NS];
   uint64_t a_full[NS], a_empty[NS];
@@ -68,20 +67,23 @@ struct Smem {
   float inv127[256];
 };
 
-template <int MODE>
-constexpr size_t smem_bytes() { return sizeof(Smem<MODE>) + 1024; }
+template <int MODE, int BM>
+constexpr size_t smem_bytes() { return sizeof(Smem<MODE, BM>) + 1024; }
 
-template <int MODE, bool DQ>
+template <int MODE, bool DQ, int BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
                   const __grid_constant__ CUtensorMap tm_tokad,   // [Mtok, RP]  bf16
                   const __grid_constant__ CUtensorMap tm_w,       // [Nout, Kc]  bf16 (MODE_BF16)
                   const __grid_constant__ CUtensorMap tm_wad,     // [Nout, RP]  bf16 (MODE_BF16)
                   const GemmArgs p) {
+  static_assert(BM % 32 == 0 && BM >= 32 && BM <= 256, "token tile");
   constexpr int NS = stages<MODE>();
+  constexpr int BMH = BM / 2;                      // tokens loaded by each CTA
+  constexpr int X_BYTES = BMH * BK * 2;
   extern __shared__ uint8_t smem_raw[];
-  Smem<MODE>& S =
-      *reinterpret_cast<Smem<MODE>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<MODE, BM>& S =
+      *reinterpret_cast<Smem<MODE, BM>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();        // 0: issues the MMAs
@@ -322,19 +324,19 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   }
 }
 
-template <int MODE, bool DQ>
-static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
-                               const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
+template <int MODE, bool DQ, int BM>
+static cudaError_t launch_pair_bm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
+                                  const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaFuncSetAttribute(k_qlora_gemm_pair<MODE, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<MODE>());
+    cudaFuncSetAttribute(k_qlora_gemm_pair<MODE, DQ, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem_bytes<MODE, BM>());
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<MODE>();
+  cfg.dynamicSmemBytes = smem_bytes<MODE, BM>();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -343,19 +345,51 @@ static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, con
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<MODE, DQ>, a0, a1, a2, a3, a);
+  return cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<MODE, DQ, BM>, a0, a1, a2, a3, a);
+}
+
+template <int BM>
+static cudaError_t launch_pair(int mode, const CUtensorMap& a0, const CUtensorMap& a1,
+                               const CUtensorMap& a2, const CUtensorMap& a3, const GemmArgs& a,
+                               int clusters, cudaStream_t s) {
+  if (mode == MODE_BF16) return launch_pair_bm<MODE_BF16, false, BM>(a0, a1, a2, a3, a, clusters, s);
+  if (a.double_quant) return launch_pair_bm<MODE_NF4, true, BM>(a0, a1, a2, a3, a, clusters, s);
+  return launch_pair_bm<MODE_NF4, false, BM>(a0, a1, a2, a3, a, clusters, s);
 }
 
 }  // namespace pair
+
+// Token-tile width of the paired GEMM for an [Mtok x Nout] output on
+// `clusters_max` SM pairs.  A pair tile costs (fixed + width) per K step --
+// the fixed part, the A-operand supply, dominates: about 4000 width units in
+// MODE_NF4 (the converter warps) and 480 in MODE_BF16 (the weight-tile TMA),
+// as timed on B200 -- and a launch lasts as many rounds as the busiest pair
+// runs tiles.  The narrower width pays only where it removes a round.
+int pair_token_tile(int mode, int64_t Mtok, int64_t Nout, int clusters_max) {
+  static const int kWidths[] = {256, 224};
+  const int64_t fixed = mode == MODE_NF4 ? 4000 : 480;
+  const int64_t n_pairs_n = (Nout + 255) / 256;
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int bm : kWidths) {
+    const int64_t tiles = n_pairs_n * ((Mtok + bm - 1) / bm);
+    const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(tiles, clusters_max));
+    const int64_t rounds = (tiles + clusters - 1) / clusters;
+    const int64_t cost = rounds * (bm + fixed);
+    if (cost < best_cost) { best_cost = cost; best = bm; }
+  }
+  return best;
+}
 
 // Paired-SM GEMM.  MODE_NF4: weights from `a` (NF4); MODE_BF16: w [Nout, Kc]
 // and wad [Nout, RP] bf16 by TMA.  Returns QLORA_OK or QLORA_ERR_CUDA.
 int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
                            const void* wad, const void* w, int RP, cudaStream_t s, int num_sms) {
   using namespace pair;
+  const int bm = pair_token_tile(mode, a.Mtok, a.Nout, num_sms / 2);
   CUtensorMap t_tok, t_tokad, t_w, t_wad;
-  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, BMH)) return QLORA_ERR_CUDA;
-  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, BMH)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, bm / 2)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, bm / 2)) return QLORA_ERR_CUDA;
   if (mode == MODE_BF16) {
     if (!make_tmap_2d_bf16(&t_w, w, a.Kc, a.Nout, a.Kc, BK, BN)) return QLORA_ERR_CUDA;
     if (!make_tmap_2d_bf16(&t_wad, wad, RP, a.Nout, RP, BK, BN)) return QLORA_ERR_CUDA;
@@ -363,12 +397,11 @@ int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const v
     t_w = t_tok;                                   // unused
     t_wad = t_tokad;
   }
-  const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + BM - 1) / BM);
+  const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + bm - 1) / bm);
   const int clusters = std::max(1, std::min(n_tiles, num_sms / 2));
   cudaError_t e;
-  if (mode == MODE_BF16) e = launch_pair<MODE_BF16, false>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
-  else if (a.double_quant) e = launch_pair<MODE_NF4, true>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
-  else e = launch_pair<MODE_NF4, false>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  if (bm == 224) e = launch_pair<224>(mode, t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  else e = launch_pair<256>(mode, t_tok, t_tokad, t_w, t_wad, a, clusters, s);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 

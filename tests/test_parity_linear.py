@@ -73,6 +73,28 @@ def test_forward_small(q, N, K, M, r, alpha, dq):
     assert rel_err(T, Tr) <= TOL
 
 
+@pytest.mark.parametrize("N,K,M,r,dq", [
+    (1024, 1024, 16, 8, False),            # decode GEMV: fewer units than SMs
+    (512, 1024, 1, 16, True),
+    (64, 4096, 3, 8, True),                # one row group split over many CTAs
+    (200, 192, 300, 16, True),             # tensor-core GEMM path
+])
+def test_forward_ignores_workspace_contents(q, N, K, M, r, dq):
+    """Every workspace byte the forward reads is written earlier in the same
+    call: a workspace full of NaN bytes changes nothing."""
+    W, X, A, B, wq = _layer(q, N, K, M, r, 16.0, seed=7000 + M, dq=dq)
+    ws = torch.full((q.workspace_bytes(1, M, N, K, r),), 0xFF, dtype=torch.uint8, device="cuda")
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    T = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+    q.qlora_linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), 16.0, Y, T, ws)
+    assert q.qlora_check_status() == 0
+    Yr, Tr = oracle.linear_fwd(X.float().numpy(), _oracle_weight(wq, W), A.float().numpy(),
+                               B.float().numpy(), 16.0, r)
+    assert torch.isfinite(Y.float()).all() and torch.isfinite(T.float()).all()
+    assert rel_err(Y, Yr) <= TOL
+    assert rel_err(T, Tr) <= TOL
+
+
 def test_forward_identity_is_exact_dequant(q):
     """X = I, A = 0: Y[m, n] = W'[n, m] exactly (one nonzero product per sum)."""
     N, K = 384, 512
