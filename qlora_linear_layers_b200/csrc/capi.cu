@@ -243,7 +243,7 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
                          static_cast<unsigned long long*>(ws), d->status, (cudaStream_t)stream,
                          d->sms);
   st = launch_status();
-  if (!st) count_launches(3);
+  if (!st) count_launches(2);
   return st;
 }
 

@@ -68,6 +68,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// The first 1024-byte-aligned address at or after a dynamic shared array,
+// reached by offsetting the array itself so the compiler keeps shared-space
+// (32-bit) addressing for everything derived from it.
+template <typename T>
+__device__ __forceinline__ T* smem_align1024(uint8_t* raw) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+  return reinterpret_cast<T*>(raw + ((1024u - (a & 1023u)) & 1023u));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -156,7 +156,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
   __shared__ __align__(16) uint32_t tbl[256 * 32];
   extern __shared__ uint8_t gsm_raw[];
   GemvSmem<NT>& S =
-      *reinterpret_cast<GemvSmem<NT>*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+      *smem_align1024<GemvSmem<NT>>(gsm_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kStages = n_stages<NT>();
   constexpr uint32_t kTx = stage_bytes<NT>();

@@ -161,17 +161,79 @@ void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float
 // ===========================================================================
 // Double quantisation
 //   1. exact per-tensor sum of absmax: histogram of 24-bit significands per
-//      fp32 exponent (integer adds: exact and order-independent);
-//   2. one thread turns the histogram into the correctly rounded fp64 sum and
+//      fp32 exponent (integer adds: exact and order-independent); the last
+//      block to finish (counted in bin 255, which no finite value uses) turns
+//      the histogram into the correctly rounded fp64 sum and
 //      mean = RN32(RN64(sum) / n);
-//   3. one warp per group of 256: d = RN32(a - mean), s = max|d|,
+//   2. one warp per group of 256: d = RN32(a - mean), s = max|d|,
 //      c = rint(RN32(RN32(d / s) * 127)).
 // ===========================================================================
 
+// Exact integer S = sum_e hist[e] * 2^(max(e,1)-1) in units of 2^-149 (a float
+// with exponent field e and significand m is m * 2^(max(e,1) - 150)), rounded
+// to the nearest double (ties to even); returns RN32(RN64(S * 2^-149) / n).
+__device__ float exact_mean(const unsigned long long* hist, int64_t n) {
+  constexpr int L = 12;                  // 384-bit accumulator, little-endian words
+  uint32_t acc[L];
+#pragma unroll
+  for (int i = 0; i < L; ++i) acc[i] = 0;
+  for (int e = 0; e < 255; ++e) {
+    const unsigned long long v = hist[e];
+    if (!v) continue;
+    const int sh = (e > 0 ? e : 1) - 1;  // 0..253
+    const int w = sh >> 5, b = sh & 31;
+    // v << b is a 96-bit number (v < 2^64, b < 32)
+    const unsigned long long lo64 = v << b;
+    const unsigned long long hi = b ? (v >> (64 - b)) : 0ull;
+    const uint32_t parts[3] = {(uint32_t)lo64, (uint32_t)(lo64 >> 32), (uint32_t)hi};
+    uint64_t carry = 0;
+    for (int k = 0; w + k < L; ++k) {
+      const uint64_t t = (uint64_t)acc[w + k] + (k < 3 ? parts[k] : 0u) + carry;
+      acc[w + k] = (uint32_t)t;
+      carry = t >> 32;
+      if (k >= 2 && carry == 0) break;
+    }
+  }
+  int tw = -1;                           // highest nonzero word
+  for (int i = L - 1; i >= 0; --i)
+    if (acc[i]) { tw = i; break; }
+  double S = 0.0;
+  if (tw >= 0) {
+    const int top = 32 * tw + 31 - __clz(acc[tw]);
+    // 64 bits of S starting at bit position lo (lo >= 0)
+    auto bits64 = [&](int lo) -> unsigned long long {
+      const int w = lo >> 5, b = lo & 31;
+      const unsigned long long w0 = acc[w];
+      const unsigned long long w1 = (w + 1 < L) ? acc[w + 1] : 0u;
+      const unsigned long long w2 = (w + 2 < L) ? acc[w + 2] : 0u;
+      const unsigned long long low = w0 | (w1 << 32);
+      return b ? ((low >> b) | (w2 << (64 - b))) : low;
+    };
+    if (top <= 52) {
+      S = ldexp((double)bits64(0), -149);             // exact
+    } else {
+      const int sh = top - 52;                         // the 53-bit significand is bits [sh, top]
+      unsigned long long mant = bits64(sh) & ((1ull << 53) - 1);
+      const uint32_t round_bit = (uint32_t)(bits64(sh - 1) & 1ull);
+      // sticky: any set bit below sh - 1
+      bool sticky = false;
+      const int below = sh - 1;                        // bits [0, below) are sticky bits
+      for (int i = 0; i < (below >> 5); ++i) sticky |= acc[i] != 0;
+      if (below & 31) sticky |= (acc[below >> 5] & ((1u << (below & 31)) - 1u)) != 0;
+      if (round_bit && (sticky || (mant & 1ull))) ++mant;
+      int expo = sh;
+      if (mant == (1ull << 53)) { mant >>= 1; ++expo; }
+      S = ldexp((double)mant, expo - 149);
+    }
+  }
+  return __double2float_rn(__ddiv_rn(S, (double)n));
+}
+
 __global__ void __launch_bounds__(256)
 k_absmax_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* __restrict__ hist,
-              int* status) {
+              float* __restrict__ mean, int* status) {
   __shared__ unsigned long long sh[256];
+  __shared__ bool last;
   for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0ull;
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -199,66 +261,19 @@ k_absmax_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* _
       atomicAdd(&sh[e], (unsigned long long)sum);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+  for (int i = threadIdx.x; i < 255; i += blockDim.x)
     if (sh[i]) atomicAdd(&hist[i], sh[i]);
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
-}
-
-// One thread: exact integer S = sum_e hist[e] * 2^(max(e,1)-1) in units of
-// 2^-149 (the value of a float with exponent field e and significand m is
-// m * 2^(max(e,1) - 150)); round S to the nearest double (ties to even), then
-// mean = RN32(RN64(S * 2^-149) / n).
-__global__ void __launch_bounds__(256)
-k_mean_finalize(const unsigned long long* __restrict__ hist_g, int64_t n,
-                float* __restrict__ mean) {
-  __shared__ unsigned long long hist[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = hist_g[i];   // parallel loads
+  // the last block to get here sums the complete histogram
+  __threadfence();
   __syncthreads();
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  constexpr int L = 12;                  // 384-bit accumulator
-  uint32_t acc[L];
-  for (int i = 0; i < L; ++i) acc[i] = 0;
-  for (int e = 0; e < 255; ++e) {
-    unsigned long long v = hist[e];
-    if (!v) continue;
-    const int sh = (e > 0 ? e : 1) - 1;  // 0..253
-    const int w = sh >> 5, b = sh & 31;
-    // v << b is a 96-bit number (v < 2^64, b < 32): low 64 bits and the
-    // bits shifted out of them
-    const unsigned long long lo64 = v << b;
-    const unsigned long long hi = b ? (v >> (64 - b)) : 0ull;
-    uint64_t carry = 0;
-    const uint32_t parts[3] = {(uint32_t)lo64, (uint32_t)(lo64 >> 32), (uint32_t)hi};
-    for (int k = 0; k < L - w; ++k) {
-      uint64_t t = (uint64_t)acc[w + k] + (k < 3 ? parts[k] : 0u) + carry;
-      acc[w + k] = (uint32_t)t;
-      carry = t >> 32;
-      if (k >= 2 && carry == 0) break;
-    }
-  }
-  int top = -1;
-  for (int i = L - 1; i >= 0 && top < 0; --i)
-    if (acc[i]) top = 32 * i + 31 - __clz(acc[i]);
-  double S;
-  if (top < 0) {
-    S = 0.0;
-  } else if (top <= 52) {
-    unsigned long long x = ((unsigned long long)acc[1] << 32) | acc[0];
-    S = ldexp((double)x, -149);                        // exact
-  } else {
-    auto bit = [&](int pos) -> uint32_t { return (acc[pos >> 5] >> (pos & 31)) & 1u; };
-    unsigned long long mant = 0;
-    for (int pos = top; pos > top - 53; --pos) mant = (mant << 1) | bit(pos);
-    const int rpos = top - 53;
-    const uint32_t round_bit = bit(rpos);
-    uint32_t sticky = 0;
-    for (int pos = rpos - 1; pos >= 0 && !sticky; --pos) sticky |= bit(pos);
-    if (round_bit && (sticky || (mant & 1ull))) ++mant;
-    int expo = top - 52;
-    if (mant == (1ull << 53)) { mant >>= 1; ++expo; }
-    S = ldexp((double)mant, expo - 149);
-  }
-  mean[0] = __double2float_rn(__ddiv_rn(S, (double)n));
+  if (threadIdx.x == 0) last = atomicAdd(&hist[255], 1ull) == (unsigned long long)gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < 255; i += blockDim.x) sh[i] = __ldcg(&hist[i]);
+  __syncthreads();
+  if (threadIdx.x == 0) mean[0] = exact_mean(sh, n);
 }
 
 __global__ void __launch_bounds__(256)
@@ -301,8 +316,7 @@ void launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, flo
                             cudaStream_t s, int num_sms) {
   cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
   int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 4);
-  k_absmax_hist<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, hist, status);
-  k_mean_finalize<<<1, 256, 0, s>>>(hist, n, dq_mean);
+  k_absmax_hist<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, hist, dq_mean, status);
   const int64_t ngroups = (n + 255) / 256;
   blocks = (int)std::min<int64_t>((ngroups + 7) / 8, (int64_t)num_sms * 8);
   k_dq_blockwise<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, dq_mean, qabsmax, dq_scale);
