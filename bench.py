@@ -174,7 +174,7 @@ def run_ours(args, rank, world, local_rank):
     from qlora_linear_layers_b200.build import build
     build()
     import qlora_linear_layers_b200 as q
-    from qlora_linear_layers_b200 import _lib, synth
+    from qlora_linear_layers_b200 import _lib, dp, synth
 
     lib = _lib.load()
     dev = torch.device("cuda", local_rank)
@@ -185,12 +185,12 @@ def run_ours(args, rank, world, local_rank):
     # ---- inputs: seeded on the host (pinned, for the end-to-end leg), then resident in HBM
     host, devt = [], []
     for p, (N, K) in enumerate(wl.weights):
-        seed_off = 100000 * rank
-        W = synth.weight(N, K, wl.seed(synth.TID_W, p) + seed_off, "bf16")
-        X = synth.activations(M, K, wl.seed(synth.TID_X, p) + seed_off)
-        A = synth.activations(r, K, wl.seed(synth.TID_A, p), sigma=0.02)
-        B = synth.activations(N, r, wl.seed(synth.TID_B, p), sigma=0.02)
-        dY = synth.activations(M, N, wl.seed(synth.TID_DY, p) + seed_off)
+        # replicated frozen weight and adapters; each rank its own tokens
+        W = synth.weight(N, K, dp.replica_seed(wl.seed(synth.TID_W, p), rank), "bf16")
+        X = synth.activations(M, K, dp.token_seed(wl.seed(synth.TID_X, p), rank))
+        A = synth.activations(r, K, dp.replica_seed(wl.seed(synth.TID_A, p), rank), sigma=0.02)
+        B = synth.activations(N, r, dp.replica_seed(wl.seed(synth.TID_B, p), rank), sigma=0.02)
+        dY = synth.activations(M, N, dp.token_seed(wl.seed(synth.TID_DY, p), rank))
         h = {k: v.pin_memory() for k, v in dict(W=W, X=X, A=A, B=B, dY=dY).items()}
         host.append(h)
         d = {k: v.to(dev) for k, v in h.items()}
@@ -251,8 +251,7 @@ def run_ours(args, rank, world, local_rank):
             q.qlora_linear_fwd(wq, d["X"][:DECODE_M], d["A"], d["B"], alpha, d["Ydec"], None, ws)
             if ev: ev[6].record(stream)
             if world > 1:
-                dist.all_reduce(d["dA"])
-                dist.all_reduce(d["dB"])
+                dp.allreduce_adapter_grads(d["dA"], d["dB"])
             if record is not None:
                 record.append((p, ev))
 
@@ -340,7 +339,7 @@ def run_ours(args, rank, world, local_rank):
     # dominant kernel: the fused NF4-dequant forward GEMM (one launch per projection)
     gemm_flops = [2 * M * N * K + 2 * M * N * r for (N, K) in wl.weights]
     achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
-    roofline = {"kernel": "k_qlora_gemm<NF4> (fused NF4-dequant forward GEMM + adapter tail)",
+    roofline = {"kernel": "k_qlora_gemm_pair<NF4> (fused NF4-dequant forward GEMM + adapter tail, paired SMs)",
                 "bound": "tensor", "achieved": achieved, "peak": tc_sus, "unit": "TFLOP/s",
                 "frac": achieved / tc_sus, "traffic": None,
                 "peak_kind": f"bf16 dense, sustained ({pk['source']})",
