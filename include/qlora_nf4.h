@@ -153,7 +153,10 @@ int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols,
  *   dq_scale device out [ceil(n_absmax/256)] fp32
  *   dq_mean  device out [1] fp32
  *   ws       device workspace of qlora_workspace_bytes(QLORA_OP_DOUBLE_QUANT, ..)
- * The mean is bit-identical for any launch order (exact integer sum).
+ * The mean is bit-identical for any launch order (exact integer sum).  One
+ * cooperative launch (all blocks co-resident, one bounded grid barrier):
+ * QLORA_ERR_CUDA if the device refuses it, QLORA_ERR_TIMEOUT in the status
+ * word if the barrier gives up.
  */
 int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
                         int8_t* qabsmax, float* dq_scale, float* dq_mean,

@@ -239,11 +239,12 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
   DeviceInfo* d = nullptr;
   int st = current_device(&d);
   if (st) return st;
-  launch_double_quantize(absmax, n_absmax, qabsmax, dq_scale, dq_mean,
-                         static_cast<unsigned long long*>(ws), d->status, (cudaStream_t)stream,
-                         d->sms);
+  const int n = launch_double_quantize(absmax, n_absmax, qabsmax, dq_scale, dq_mean,
+                                       static_cast<unsigned long long*>(ws), d->status,
+                                       (cudaStream_t)stream, d->sms);
   st = launch_status();
-  if (!st) count_launches(2);
+  if (!st && n < 0) st = QLORA_ERR_CUDA;
+  if (!st) count_launches(n);
   return st;
 }
 

@@ -49,14 +49,12 @@ namespace eng {
 constexpr int BN = 128;          // weight-side rows per tile (MMA M)
 constexpr int BM = 256;          // tokens per tile (MMA N)
 constexpr int BK = 64;           // contraction per stage (= one NF4 block)
-constexpr int MAX_NA = 2;        // adapter K steps (r <= 128)
 constexpr int X_BYTES = BM * BK * 2;            // 32 KB token tile
 constexpr int W_BYTES = BN * BK * 2;            // 16 KB weight tile
 constexpr int ACC_COL = 0;                      // accumulator: TMEM columns [0, 256)
 constexpr int A_COL = 256;                      // NF4 A ring: stages x 32 columns
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 448;                // 14 warps
-constexpr int EPI_WARP0 = 2;                    // warps 2-5: epilogue
 constexpr int CVT_WARP0 = 6;                    // warps 6-13: converters
 
 // Pipeline depth.  MODE_NF4 keeps only token tiles in shared memory (the

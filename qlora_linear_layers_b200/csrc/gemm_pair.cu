@@ -48,7 +48,6 @@ constexpr int ACC_COL = 0;                       // accumulator: TMEM columns [0
 constexpr int A_COL = 256;                       // MODE_NF4 A ring: 8 x 32 columns
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 448;                 // 14 warps
-constexpr int EPI_WARP0 = 2;                     // warps 2-5: epilogue
 constexpr int CVT_WARP0 = 6;                     // warps 6-13: A-operand producers
 constexpr uint16_t kBoth = 0x3;                  // cluster CTA mask of the pair
 

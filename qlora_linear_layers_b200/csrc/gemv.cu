@@ -121,10 +121,6 @@ __host__ __device__ __forceinline__ int n_pieces(int rgp, int spr, int64_t U, in
   return (int)(owner_cta((int64_t)rgp * spr + spr - 1, U, P) - owner_cta((int64_t)rgp * spr, U, P) + 1);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" :: "n"(kCW * 32) : "memory");
 }

@@ -11,7 +11,8 @@ namespace qnf4 {
 void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
                      int* status, cudaStream_t s, int num_sms);
 
-void launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
+// One cooperative kernel; returns the kernels launched (1), -1 if refused.
+int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
                             float* dq_mean, unsigned long long* hist, int* status,
                             cudaStream_t s, int num_sms);
 

@@ -159,53 +159,67 @@ void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float
 }
 
 // ===========================================================================
-// Double quantisation
+// Double quantisation, one cooperative kernel:
 //   1. exact per-tensor sum of absmax: histogram of 24-bit significands per
-//      fp32 exponent (integer adds: exact and order-independent); the last
-//      block to finish (counted in bin 255, which no finite value uses) turns
-//      the histogram into the correctly rounded fp64 sum and
-//      mean = RN32(RN64(sum) / n);
-//   2. one warp per group of 256: d = RN32(a - mean), s = max|d|,
-//      c = rint(RN32(RN32(d / s) * 127)).
+//      fp32 exponent (integer adds: exact and order-independent), per block
+//      in shared memory, then added into a global histogram;
+//   2. one grid barrier (counted in bin 255, which no finite value uses);
+//      every block turns the complete histogram into the correctly rounded
+//      fp64 sum and mean = RN32(RN64(sum) / n) -- the same bits everywhere;
+//   3. one warp per group of 256: d = RN32(a - mean), s = max|d|,
+//      c = rint(RN32(RN32(d / s) * 127)) (the group re-read from L2).
 // ===========================================================================
 
 // Exact integer S = sum_e hist[e] * 2^(max(e,1)-1) in units of 2^-149 (a float
 // with exponent field e and significand m is m * 2^(max(e,1) - 150)), rounded
 // to the nearest double (ties to even); returns RN32(RN64(S * 2^-149) / n).
-__device__ float exact_mean(const unsigned long long* hist, int64_t n) {
-  constexpr int L = 12;                  // 384-bit accumulator, little-endian words
-  uint32_t acc[L];
-#pragma unroll
-  for (int i = 0; i < L; ++i) acc[i] = 0;
-  for (int e = 0; e < 255; ++e) {
-    const unsigned long long v = hist[e];
-    if (!v) continue;
-    const int sh = (e > 0 ? e : 1) - 1;  // 0..253
-    const int w = sh >> 5, b = sh & 31;
-    // v << b is a 96-bit number (v < 2^64, b < 32)
-    const unsigned long long lo64 = v << b;
-    const unsigned long long hi = b ? (v >> (64 - b)) : 0ull;
-    const uint32_t parts[3] = {(uint32_t)lo64, (uint32_t)(lo64 >> 32), (uint32_t)hi};
-    uint64_t carry = 0;
-    for (int k = 0; w + k < L; ++k) {
-      const uint64_t t = (uint64_t)acc[w + k] + (k < 3 ? parts[k] : 0u) + carry;
-      acc[w + k] = (uint32_t)t;
-      carry = t >> 32;
-      if (k >= 2 && carry == 0) break;
+// Called by one full warp: lane w < 12 sums the bins whose shift falls in
+// 32-bit word w as a 128-bit integer (at most 32 terms below 2^95), then lane
+// 0 carries the words into a 384-bit integer and rounds it.  Every lane
+// returns the result.
+__device__ float exact_mean_warp(const unsigned long long* hist, int64_t n) {
+  constexpr int L = 12;                  // 384-bit integer, little-endian 32-bit words
+  const int lane = threadIdx.x & 31;
+  unsigned __int128 part = 0;
+  if (lane < L) {
+    // bins with shift sh = max(e,1) - 1 in [32 lane, 32 lane + 31]
+    const int e_lo = lane == 0 ? 0 : 32 * lane + 1;
+    const int e_hi = min(32 * lane + 32, 254);
+    for (int e = e_lo; e <= e_hi; ++e) {
+      const unsigned long long v = hist[e];
+      const int sh = (e > 0 ? e : 1) - 1;
+      part += (unsigned __int128)v << (sh & 31);
     }
   }
-  int tw = -1;                           // highest nonzero word
-  for (int i = L - 1; i >= 0; --i)
-    if (acc[i]) { tw = i; break; }
+  uint32_t acc[L];
+  unsigned __int128 carry = 0;
+#pragma unroll
+  for (int w = 0; w < L; ++w) {
+    unsigned __int128 pw = 0;
+    const uint64_t lo = __shfl_sync(0xffffffffu, (uint64_t)part, w);
+    const uint64_t hi = __shfl_sync(0xffffffffu, (uint64_t)(part >> 64), w);
+    pw = ((unsigned __int128)hi << 64) | lo;
+    const unsigned __int128 t = pw + carry;
+    acc[w] = (uint32_t)t;
+    carry = t >> 32;
+  }
+  // word i of S, branch-free (i may be out of range: 0)
+  auto word = [&](int i) -> uint32_t {
+    uint32_t r = 0;
+#pragma unroll
+    for (int w = 0; w < L; ++w) r = (i == w) ? acc[w] : r;
+    return r;
+  };
+  int tw = -1;
+#pragma unroll
+  for (int w = 0; w < L; ++w) tw = acc[w] ? w : tw;
   double S = 0.0;
   if (tw >= 0) {
-    const int top = 32 * tw + 31 - __clz(acc[tw]);
+    const int top = 32 * tw + 31 - __clz(word(tw));
     // 64 bits of S starting at bit position lo (lo >= 0)
     auto bits64 = [&](int lo) -> unsigned long long {
       const int w = lo >> 5, b = lo & 31;
-      const unsigned long long w0 = acc[w];
-      const unsigned long long w1 = (w + 1 < L) ? acc[w + 1] : 0u;
-      const unsigned long long w2 = (w + 2 < L) ? acc[w + 2] : 0u;
+      const unsigned long long w0 = word(w), w1 = word(w + 1), w2 = word(w + 2);
       const unsigned long long low = w0 | (w1 << 32);
       return b ? ((low >> b) | (w2 << (64 - b))) : low;
     };
@@ -216,10 +230,14 @@ __device__ float exact_mean(const unsigned long long* hist, int64_t n) {
       unsigned long long mant = bits64(sh) & ((1ull << 53) - 1);
       const uint32_t round_bit = (uint32_t)(bits64(sh - 1) & 1ull);
       // sticky: any set bit below sh - 1
+      const int below = sh - 1;
       bool sticky = false;
-      const int below = sh - 1;                        // bits [0, below) are sticky bits
-      for (int i = 0; i < (below >> 5); ++i) sticky |= acc[i] != 0;
-      if (below & 31) sticky |= (acc[below >> 5] & ((1u << (below & 31)) - 1u)) != 0;
+#pragma unroll
+      for (int w = 0; w < L; ++w) {
+        const uint32_t m = (32 * w + 32 <= below) ? 0xFFFFFFFFu
+                         : (32 * w < below) ? ((1u << (below - 32 * w)) - 1u) : 0u;
+        sticky |= (acc[w] & m) != 0;
+      }
       if (round_bit && (sticky || (mant & 1ull))) ++mant;
       int expo = sh;
       if (mant == (1ull << 53)) { mant >>= 1; ++expo; }
@@ -229,68 +247,100 @@ __device__ float exact_mean(const unsigned long long* hist, int64_t n) {
   return __double2float_rn(__ddiv_rn(S, (double)n));
 }
 
-__global__ void __launch_bounds__(256)
-k_absmax_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* __restrict__ hist,
-              float* __restrict__ mean, int* status) {
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(512)
+k_double_quant(const float* __restrict__ absmax, int64_t n, unsigned long long* __restrict__ hist,
+               int8_t* __restrict__ qabsmax, float* __restrict__ dq_scale, float* __restrict__ mean,
+               int* status) {
   __shared__ unsigned long long sh[256];
-  __shared__ bool last;
+  __shared__ float s_mu;
+  __shared__ int s_ok;
   for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0ull;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   bool bad = false;
+  // ---- 1. histogram; every lane of a warp runs the same number of
+  // iterations (match/reduce below need the full warp).  A thread's kU loads
+  // are all issued before the first is used.
+  constexpr int kU = 16;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // every lane of a warp runs the same number of iterations (match/reduce
-  // below need the full warp)
   const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  for (int64_t base = first; base < n; base += stride) {
-    const int64_t i = base + lane;
-    uint32_t e = 0xFFFFFFFFu, mant = 0;
-    if (i < n) {
-      const uint32_t u = __float_as_uint(absmax[i]);
-      if (u >= 0x7F800000u) {          // negative (sign set, nonzero) or NaN/Inf
-        if (u != 0x80000000u) bad = true;
-      } else {
-        e = u >> 23;
-        mant = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-      }
+  for (int64_t base0 = first; base0 < n; base0 += kU * stride) {
+    uint32_t u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int64_t i = base0 + k * stride + lane;
+      u[k] = i < n ? __float_as_uint(__ldcs(absmax + i)) : 0xFFFFFFFFu;   // sentinel: no element
     }
-    const uint32_t grp = __match_any_sync(0xffffffffu, e);
-    const uint32_t sum = __reduce_add_sync(grp, mant);       // < 32 * 2^24
-    const int leader = __ffs(grp) - 1;
-    if (lane == leader && e != 0xFFFFFFFFu && sum)
-      atomicAdd(&sh[e], (unsigned long long)sum);
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      if (base0 + k * stride >= n) break;        // warp-uniform
+      uint32_t e = 0xFFFFFFFFu, mant = 0;
+      if (u[k] != 0xFFFFFFFFu) {
+        if (u[k] >= 0x7F800000u) {     // negative (sign set, nonzero) or NaN/Inf
+          if (u[k] != 0x80000000u) bad = true;
+        } else {
+          e = u[k] >> 23;
+          mant = (u[k] & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+        }
+      }
+      const uint32_t grp = __match_any_sync(0xffffffffu, e);
+      const uint32_t sum = __reduce_add_sync(grp, mant);     // < 32 * 2^24
+      const int leader = __ffs(grp) - 1;
+      if (lane == leader && e != 0xFFFFFFFFu && sum)
+        atomicAdd(&sh[e], (unsigned long long)sum);
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < 255; i += blockDim.x)
     if (sh[i]) atomicAdd(&hist[i], sh[i]);
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
-  // the last block to get here sums the complete histogram
+  // ---- 2. grid barrier (all blocks are co-resident: cooperative launch),
+  // bounded; then the exact mean from the complete histogram
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&hist[255], 1ull) == (unsigned long long)gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    atomicAdd(&hist[255], 1ull);
+    int ok = 1;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_u64(&hist[255]) < (unsigned long long)gridDim.x) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        ok = 0;
+        set_status(status, QLORA_ERR_TIMEOUT);
+        break;
+      }
+    }
+    s_ok = ok;
+  }
   __syncthreads();
-  if (!last) return;
-  __threadfence();
+  if (!s_ok) return;
   for (int i = threadIdx.x; i < 255; i += blockDim.x) sh[i] = __ldcg(&hist[i]);
   __syncthreads();
-  if (threadIdx.x == 0) mean[0] = exact_mean(sh, n);
-}
-
-__global__ void __launch_bounds__(256)
-k_dq_blockwise(const float* __restrict__ absmax, int64_t n, const float* __restrict__ mean,
-               int8_t* __restrict__ qabsmax, float* __restrict__ dq_scale) {
-  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    const float mu = exact_mean_warp(sh, n);
+    if (threadIdx.x == 0) {
+      s_mu = mu;
+      if (blockIdx.x == 0) mean[0] = mu;
+    }
+  }
+  __syncthreads();
+  // ---- 3. one warp per group of 256
+  const float mu = s_mu;
   const int64_t ngroups = (n + 255) / 256;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const float mu = mean[0];
   for (int64_t g = warp; g < ngroups; g += nwarps) {
     float d[8];
     float m = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t i = g * 256 + j * 32 + lane;
-      d[j] = (i < n) ? __fsub_rn(absmax[i], mu) : 0.0f;
+      d[j] = (i < n) ? __fsub_rn(__ldcg(absmax + i), mu) : 0.0f;
       m = fmaxf(m, fabsf(d[j]));
     }
 #pragma unroll
@@ -311,15 +361,18 @@ k_dq_blockwise(const float* __restrict__ absmax, int64_t n, const float* __restr
   }
 }
 
-void launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
-                            float* dq_mean, unsigned long long* hist, int* status,
-                            cudaStream_t s, int num_sms) {
+// Returns the number of kernels launched (1), or -1 if the cooperative launch
+// was refused.
+int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
+                           float* dq_mean, unsigned long long* hist, int* status,
+                           cudaStream_t s, int num_sms) {
   cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
-  int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 4);
-  k_absmax_hist<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, hist, dq_mean, status);
-  const int64_t ngroups = (n + 255) / 256;
-  blocks = (int)std::min<int64_t>((ngroups + 7) / 8, (int64_t)num_sms * 8);
-  k_dq_blockwise<<<std::max(blocks, 1), 256, 0, s>>>(absmax, n, dq_mean, qabsmax, dq_scale);
+  // one wide block per SM (fewer blocks meet on the few busy histogram bins)
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 8191) / 8192, (int64_t)num_sms));
+  void* args[] = {(void*)&absmax, (void*)&n, (void*)&hist, (void*)&qabsmax, (void*)&dq_scale,
+                  (void*)&dq_mean, (void*)&status};
+  return cudaLaunchCooperativeKernel((const void*)k_double_quant, dim3(blocks), dim3(512), args, 0, s) ==
+                 cudaSuccess ? 1 : -1;
 }
 
 // ===========================================================================
