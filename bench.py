@@ -224,36 +224,39 @@ def run_ours(args, rank, world, local_rank):
     comps = ("quantize", "double_quant", "dequantize", "fwd", "bwd", "decode")
     stream = torch.cuda.current_stream()
 
+    def step_proj(p, d, record, gemm_ev):
+        wq = d["wq"]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if record is not None else None
+        if ev: ev[0].record(stream)
+        q.nf4_quantize(d["W"], wq.packed, wq.absmax)
+        if ev: ev[1].record(stream)
+        q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws)
+        if ev: ev[2].record(stream)
+        q.nf4_dequantize(wq, d["Wdeq"])
+        if ev: ev[3].record(stream)
+        if gemm_ev is not None:
+            g0, g1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            # torch creates the CUDA event on first record; the library's
+            # record at the GEMM launch supersedes this one
+            g0.record(stream)
+            g1.record(stream)
+            lib.qlora_profile_gemm_events(g0.cuda_event, g1.cuda_event)
+            gemm_ev.append((p, g0, g1))
+        q.qlora_linear_fwd(wq, d["X"], d["A"], d["B"], alpha, d["Y"], d["T"], ws)
+        if ev: ev[4].record(stream)
+        q.qlora_linear_bwd(wq, d["X"], d["dY"], d["A"], d["B"], alpha, d["dX"], d["dA"], d["dB"],
+                           T=d["T"], ws=ws)
+        if ev: ev[5].record(stream)
+        q.qlora_linear_fwd(wq, d["X"][:DECODE_M], d["A"], d["B"], alpha, d["Ydec"], None, ws)
+        if ev: ev[6].record(stream)
+        if world > 1:
+            dp.allreduce_adapter_grads(d["dA"], d["dB"])
+        if record is not None:
+            record.append((p, ev))
+
     def step(record, gemm_ev):
         for p, d in enumerate(devt):
-            wq = d["wq"]
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if record is not None else None
-            if ev: ev[0].record(stream)
-            q.nf4_quantize(d["W"], wq.packed, wq.absmax)
-            if ev: ev[1].record(stream)
-            q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws)
-            if ev: ev[2].record(stream)
-            q.nf4_dequantize(wq, d["Wdeq"])
-            if ev: ev[3].record(stream)
-            if gemm_ev is not None:
-                g0, g1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
-                # torch creates the CUDA event on first record; the library's
-                # record at the GEMM launch supersedes this one
-                g0.record(stream)
-                g1.record(stream)
-                lib.qlora_profile_gemm_events(g0.cuda_event, g1.cuda_event)
-                gemm_ev.append((p, g0, g1))
-            q.qlora_linear_fwd(wq, d["X"], d["A"], d["B"], alpha, d["Y"], d["T"], ws)
-            if ev: ev[4].record(stream)
-            q.qlora_linear_bwd(wq, d["X"], d["dY"], d["A"], d["B"], alpha, d["dX"], d["dA"], d["dB"],
-                               T=d["T"], ws=ws)
-            if ev: ev[5].record(stream)
-            q.qlora_linear_fwd(wq, d["X"][:DECODE_M], d["A"], d["B"], alpha, d["Ydec"], None, ws)
-            if ev: ev[6].record(stream)
-            if world > 1:
-                dp.allreduce_adapter_grads(d["dA"], d["dB"])
-            if record is not None:
-                record.append((p, ev))
+            step_proj(p, d, record, gemm_ev)
 
     def timed(nsteps, body):
         if world > 1:
@@ -353,17 +356,34 @@ def run_ours(args, rank, world, local_rank):
         h2d = sum(h[k].numel() * h[k].element_size() for h in host for k in ("W", "X", "A", "B", "dY"))
         d2h = sum(h[k].numel() * h[k].element_size() for h in host for k in ("dA_out", "dB_out"))
 
+        # Each step copies every projection's inputs from pinned host memory on
+        # a copy stream; a projection's compute waits for its own copies only,
+        # and the next step's copies into a projection's buffers wait for the
+        # compute that read them.  dA and dB are read back every step.
+        copy_stream = torch.cuda.Stream(device=dev)
+        ready = [torch.cuda.Event() for _ in devt]
+        done = [torch.cuda.Event() for _ in devt]
+        for e in done:
+            e.record(stream)
+
         def e2e_step():
-            for h, d in zip(host, devt):
-                for k in ("W", "X", "A", "B", "dY"):
-                    d[k].copy_(h[k], non_blocking=True)
-            step(None, None)
-            for h, d in zip(host, devt):
+            for p, (h, d) in enumerate(zip(host, devt)):
+                copy_stream.wait_event(done[p])
+                with torch.cuda.stream(copy_stream):
+                    for k in ("W", "X", "A", "B", "dY"):
+                        d[k].copy_(h[k], non_blocking=True)
+                ready[p].record(copy_stream)
+            for p, (h, d) in enumerate(zip(host, devt)):
+                stream.wait_event(ready[p])
+                step_proj(p, d, None, None)
+                done[p].record(stream)
                 h["dA_out"].copy_(d["dA"], non_blocking=True)
                 h["dB_out"].copy_(d["dB"], non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
+        for e in done:
+            e.record(stream)
         e_ms = timed(args.steps, e2e_step)
         e2e = {"value": step_flops * world / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
