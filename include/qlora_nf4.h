@@ -70,7 +70,9 @@ typedef enum {
  *
  *   packed   [rows*cols/2]  two codes per byte, element 2j in the HIGH nibble
  *   absmax   [rows*cols/64] fp32 block scales      (used when double_quant == 0)
- *   qabsmax  [rows*cols/64] int8 block-scale codes (used when double_quant == 1)
+ *   qabsmax  [rows*cols/64] int8 block-scale codes in [-127, 127], as
+ *            nf4_double_quantize writes them (used when double_quant == 1;
+ *            -128 is outside the format)
  *   dq_scale [ceil(rows*cols/64/256)] fp32 group scales (double_quant == 1)
  *   dq_mean  [1] fp32 per-tensor mean offset, device     (double_quant == 1)
  *
