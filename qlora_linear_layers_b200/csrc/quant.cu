@@ -16,47 +16,23 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise: one thread owns 8 consecutive weights (one 16-byte bf16 load, a
-// 4-byte code store), 8 adjacent lanes own one 64-weight block, so every warp
-// access is contiguous.  absmax is an integer max over |w| bit patterns
-// (exact; NaN/Inf show up as >= 0x7f800000), joined by 3 shuffles.
+// Quantise: one thread owns one 64-weight block (eight 16-byte bf16 loads or
+// sixteen fp32 ones, a 32-byte code store and its absmax), so the block max,
+// the reciprocal and the stores cost one thread's work per 64 weights.
+// absmax is an integer max over |w| bit patterns (exact; NaN/Inf show up as
+// >= 0x7f800000).
 //
-// Code of x = RN32(w / a):  x' = RN32(w * RN32(1/a)) is within 2.5 ulp of x.
-// A 64-entry bucket table over [-1, 1] (width 1/16, index = round(16 x + 16),
-// read with one 8-byte shared load) holds the single threshold T that can
-// fall in the bucket and the number of thresholds below it.  When x' is more
-// than 8 ulp from T, x and x' are on the same side of every threshold and the
-// code is base + (x' >= T); otherwise -- and for blocks whose absmax is 0 or
-// below 2^-125 -- x is computed exactly with the IEEE division (a rarely
-// taken branch, kept out of the unrolled loop).  Thresholds sit >= 1e-4 from bucket edges (checked on the
-// host), so x' may pick the neighbouring bucket near an edge without effect.
+// Code of x = RN32(w / a):  x' = RN32(w * rcp(a)) with the hardware reciprocal
+// (at most 1 ulp off) is within 3.5 ulp of x.  A 64-entry bucket table over
+// [-1, 1] (width 1/16, index = round(16 x + 16), read with one 8-byte shared
+// load) holds the single threshold T that can fall in the bucket and the
+// number of thresholds below it.  When x' is more than 8 ulp from T, x and x'
+// are on the same side of every threshold and the code is base + (x' >= T);
+// a block with any x' within 8 ulp of its T -- or whose absmax is 0 or below
+// 2^-125 -- is redone with the IEEE division (rare; out of line).  Thresholds
+// sit >= 1e-4 from bucket edges (checked on the host), so x' may pick the
+// neighbouring bucket near an edge without effect.
 // ===========================================================================
-
-// Loaders return the 8 weights as fp32 bit patterns and the max of their
-// magnitudes' bit patterns (bf16: a 16-bit SIMD max over packed pairs).
-template <typename T> struct Loader8;
-template <> struct Loader8<__nv_bfloat16> {
-  __device__ __forceinline__ static uint32_t load(const void* base, int64_t chunk, uint32_t (&u)[8]) {
-    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(base) + chunk);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t mp = __vmaxu2(__vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
-                           __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
-#pragma unroll
-    for (int j = 0; j < 4; ++j) { u[2 * j] = w[j] << 16; u[2 * j + 1] = w[j] & 0xFFFF0000u; }
-    return max(mp << 16, mp & 0xFFFF0000u);
-  }
-};
-template <> struct Loader8<float> {
-  __device__ __forceinline__ static uint32_t load(const void* base, int64_t chunk, uint32_t (&u)[8]) {
-    const uint4* p = reinterpret_cast<const uint4*>(base) + 2 * chunk;
-    const uint4 a = __ldcs(p), b = __ldcs(p + 1);
-    u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w; u[4] = b.x; u[5] = b.y; u[6] = b.z; u[7] = b.w;
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = max(m, u[i] & 0x7FFFFFFFu);
-    return m;
-  }
-};
 
 struct Bucket { float thr; uint32_t base; };
 
@@ -65,30 +41,66 @@ __device__ __forceinline__ uint32_t bucket_index(float x) {
   return __float_as_uint(fmaf(x, 16.0f, 8388624.0f)) & 63u;
 }
 
-// Exact codes x = RN32(w / a) for the elements of `chunk` flagged in `mask`
-// (rare: a fast quotient within 8 ulp of a threshold, or a zero / tiny absmax
-// block).  The flagged weights are re-read (cached) rather than passed in, so
-// the hot loop keeps its values in registers.
+__device__ __forceinline__ float rcp_approx(float a) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(a));
+  return r;
+}
+
+// Weight i (0..63) of a block as an fp32 bit pattern, from the block's words.
+template <typename T> struct BlockWords;
+template <> struct BlockWords<__nv_bfloat16> {
+  static constexpr int kWords = 32;               // bf16 pairs, element 2j in the low half
+  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) {
+    return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
+  }
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+    return max(m << 16, m & 0xFFFF0000u);
+  }
+};
+template <> struct BlockWords<float> {
+  static constexpr int kWords = 64;
+  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) { return w[i]; }
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) m = max(m, w[j] & 0x7FFFFFFFu);
+    return m;
+  }
+};
+
+// Exact codes of block `blk` (x = RN32(w / a), or 0 for a zero block),
+// written straight to `packed`: the rare path, kept out of line so the hot
+// loop keeps its registers.
 template <typename T>
-__device__ __noinline__ uint32_t exact_codes(const void* W, int64_t chunk, float a, bool zero_block,
-                                             uint32_t mask, uint32_t out, const Bucket* bks) {
-  for (int i = 0; i < 8; ++i) {
-    if (!((mask >> i) & 1u)) continue;
+__device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float a, bool zero_block,
+                                               const Bucket* bks, uint8_t* packed) {
+  uint32_t out[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = 0u;
+  for (int i = 0; i < 64; ++i) {
     float w;
-    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[chunk * 8 + i]);
-    else w = reinterpret_cast<const float*>(W)[chunk * 8 + i];
+    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[blk * 64 + i]);
+    else w = reinterpret_cast<const float*>(W)[blk * 64 + i];
     const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
     const Bucket bk = bks[bucket_index(x)];
     const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
-    const int sh = 8 * (i >> 1) + ((i & 1) ? 0 : 4);
-    out = (out & ~(0xFu << sh)) | (code << sh);
+    const int sh = 8 * ((i >> 1) & 3) + ((i & 1) ? 0 : 4);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k == (i >> 3)) out[k] |= code << sh;
   }
-  return out;
+  uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256)
-k_nf4_quantize(const void* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ packed,
+k_nf4_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
                float* __restrict__ absmax, Nf4Tables tb, int* status) {
   __shared__ Bucket s_bk[64];
   if (threadIdx.x < 64) {
@@ -97,65 +109,63 @@ k_nf4_quantize(const void* __restrict__ W, int64_t nchunks, uint8_t* __restrict_
     s_bk[b].base = tb.bucket_base[b];
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  constexpr int kWords = BlockWords<T>::kWords;
   bool bad = false;
-  // Two chunks per iteration (both loads in flight before either is used);
-  // every lane of a warp runs the same number of iterations (shuffles below).
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nchunks;
-       base += 2 * stride) {
-    uint32_t u[2][8], mloc[2] = {0u, 0u};
-    int64_t chunk[2];
-    bool active[2];
+  for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
+       blk += (int64_t)gridDim.x * blockDim.x) {
+    uint32_t w[kWords];
+    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * blk;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      chunk[h] = base + h * stride + lane;
-      active[h] = chunk[h] < nchunks;             // whole 8-lane groups (nchunks % 8 == 0)
-      if (active[h]) mloc[h] = Loader8<T>::load(W, chunk[h], u[h]);
+    for (int k = 0; k < kWords / 4; ++k) {
+      const uint4 v = __ldg(src + k);
+      w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
     }
+    uint32_t m = BlockWords<T>::absmax_bits(w);
+    if (m >= 0x7F800000u) { bad = true; m = 0; }
+    const float a = __uint_as_float(m);
+    const bool exact_block = m < 0x01000000u;     // a == 0 or a < 2^-125
+    const float inv = exact_block ? 0.0f : rcp_approx(a);
+    uint32_t out[8];
+    uint32_t nearm = 0xFFFFFFFFu;                 // min over the block of (ulp distance to T) + 8
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t m = mloc[h];
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      if (!active[h]) continue;
-      if (m >= 0x7F800000u) { bad = true; m = 0; }
-      const float a = __uint_as_float(m);
-      const bool exact_block = m < 0x01000000u;   // a == 0 or a < 2^-125
-      const float inv = exact_block ? 0.0f : __frcp_rn(a);
-      uint32_t out = 0;
-      bool anynear = exact_block;
+    for (int k = 0; k < 8; ++k) {
+      uint32_t o = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float x = __fmul_rn(__uint_as_float(u[h][i]), inv);
+      for (int e = 0; e < 8; ++e) {
+        const int i = 8 * k + e;
+        const float x = __fmul_rn(__uint_as_float(BlockWords<T>::elem(w, i)), inv);
         const Bucket bk = s_bk[bucket_index(x)];
-        // within 8 ulp of the threshold (same sign there, so the bit patterns
-        // differ by the ulp distance): decide exactly below
-        anynear |= (uint32_t)(__float_as_int(x) - __float_as_int(bk.thr) + 8) <= 16u;
+        // same sign near T, so the bit patterns differ by the ulp distance
+        nearm = min(nearm, (uint32_t)(__float_as_int(x) - __float_as_int(bk.thr) + 8));
         const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
-        // element 2j -> high nibble of byte j; byte j at bits 8j (fields disjoint: add = or)
-        out += code << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
+        // element 2j -> high nibble of byte j (fields disjoint: add = or)
+        o += code << (8 * (e >> 1) + ((e & 1) ? 0 : 4));
       }
-      if (anynear) out = exact_codes<T>(W, chunk[h], a, m == 0, 0xFFu, out, s_bk);
-      reinterpret_cast<uint32_t*>(packed)[chunk[h]] = out;
-      if ((lane & 7) == 0) absmax[chunk[h] >> 3] = a;
+      out[k] = o;
     }
+    if (exact_block || nearm <= 16u) {
+      exact_block_codes<T>(W, blk, a, m == 0, s_bk, packed);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
+      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    absmax[blk] = a;
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
 }
 
 void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
                      int* status, cudaStream_t s, int num_sms) {
-  const int64_t nchunks = n / 8;
+  const int64_t nblk = n / 64;
   const int threads = 256;
-  int blocks = (int)std::min<int64_t>((nchunks + threads - 1) / threads, (int64_t)num_sms * 8);
+  int blocks = (int)std::min<int64_t>((nblk + threads - 1) / threads, (int64_t)num_sms * 8);
   blocks = std::max(blocks, 1);
   const Nf4Tables& tb = host_tables();
   if (dtype == QLORA_BF16)
-    k_nf4_quantize<__nv_bfloat16><<<blocks, threads, 0, s>>>(W, nchunks, packed, absmax, tb, status);
+    k_nf4_quantize<__nv_bfloat16><<<blocks, threads, 0, s>>>(W, nblk, packed, absmax, tb, status);
   else
-    k_nf4_quantize<float><<<blocks, threads, 0, s>>>(W, nchunks, packed, absmax, tb, status);
+    k_nf4_quantize<float><<<blocks, threads, 0, s>>>(W, nblk, packed, absmax, tb, status);
 }
 
 // ===========================================================================
