@@ -24,9 +24,10 @@ namespace qnf4 {
 //
 // Code of x = RN32(w / a):  x' = RN32(w * rcp(a)) with the hardware reciprocal
 // (at most 1 ulp off) is within 3.5 ulp of x.  A 64-entry bucket table over
-// [-1, 1] (width 1/16, index = round(16 x + 16), read with one 8-byte shared
-// load) holds the single threshold T that can fall in the bucket and the
-// number of thresholds below it.  When x' is more than 8 ulp from T, x and x'
+// [-1, 1] (width 1/16, index = round(16 x + 16), one 8-byte shared load from
+// a copy per lane, so the 32 lanes never meet on a bank) holds the single
+// threshold T that can fall in the bucket and the number of thresholds below
+// it.  When x' is more than 8 ulp from T, x and x'
 // are on the same side of every threshold and the code is base + (x' >= T);
 // a block with any x' within 8 ulp of its T -- or whose absmax is 0 or below
 // 2^-125 -- is redone with the IEEE division (rare; out of line).  Thresholds
@@ -86,7 +87,7 @@ __device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float
     if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[blk * 64 + i]);
     else w = reinterpret_cast<const float*>(W)[blk * 64 + i];
     const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
-    const Bucket bk = bks[bucket_index(x)];
+    const Bucket bk = bks[bucket_index(x) * 32];
     const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
     const int sh = 8 * ((i >> 1) & 3) + ((i & 1) ? 0 : 4);
 #pragma unroll
@@ -102,13 +103,13 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 k_nf4_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
                float* __restrict__ absmax, Nf4Tables tb, int* status) {
-  __shared__ Bucket s_bk[64];
-  if (threadIdx.x < 64) {
-    const int b = threadIdx.x;
-    s_bk[b].thr = tb.bucket_thr[b];
-    s_bk[b].base = tb.bucket_base[b];
+  __shared__ Bucket s_bk[64 * 32];               // bucket b, lane l at b * 32 + l
+  for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
+    s_bk[i].thr = tb.bucket_thr[i >> 5];
+    s_bk[i].base = tb.bucket_base[i >> 5];
   }
   __syncthreads();
+  const Bucket* bk_lane = s_bk + (threadIdx.x & 31);
   constexpr int kWords = BlockWords<T>::kWords;
   bool bad = false;
   for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
@@ -134,7 +135,7 @@ k_nf4_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ p
       for (int e = 0; e < 8; ++e) {
         const int i = 8 * k + e;
         const float x = __fmul_rn(__uint_as_float(BlockWords<T>::elem(w, i)), inv);
-        const Bucket bk = s_bk[bucket_index(x)];
+        const Bucket bk = bk_lane[bucket_index(x) * 32];
         // same sign near T, so the bit patterns differ by the ulp distance
         nearm = min(nearm, (uint32_t)(__float_as_int(x) - __float_as_int(bk.thr) + 8));
         const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
@@ -159,7 +160,8 @@ void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float
                      int* status, cudaStream_t s, int num_sms) {
   const int64_t nblk = n / 64;
   const int threads = 256;
-  int blocks = (int)std::min<int64_t>((nblk + threads - 1) / threads, (int64_t)num_sms * 8);
+  // one block per thread: other CTAs' loads cover each block's compute
+  int blocks = (int)std::min<int64_t>((nblk + threads - 1) / threads, (int64_t)1 << 30);
   blocks = std::max(blocks, 1);
   const Nf4Tables& tb = host_tables();
   if (dtype == QLORA_BF16)
