@@ -43,6 +43,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA NF4 linear TFLOP/s & quant/dequant GB/s, % of B200 roofline"
+# DRAM bytes (read + write) per launch of the fused forward GEMM on this
+# workload, averaged over the step's three launches (gate, up: 364.9 MB each;
+# down: 653.2 MB), from one ncu capture of each shape (dram__bytes_read.sum +
+# dram__bytes_write.sum of `bench.py --case fwd --tokens 8192 --proj 0|2`).
+# The algorithmic bytes are 407 MB per launch.
+FWD_GEMM_DRAM_BYTES_PER_LAUNCH = (2 * 364877568 + 653239040) / 3
 WORKLOAD = "mlp_7b"
 DECODE_M = 16
 
@@ -344,7 +350,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     roofline = {"kernel": "k_qlora_gemm_pair<NF4> (fused NF4-dequant forward GEMM + adapter tail, paired SMs)",
                 "bound": "tensor", "achieved": achieved, "peak": tc_sus, "unit": "TFLOP/s",
-                "frac": achieved / tc_sus, "traffic": None,
+                "frac": achieved / tc_sus, "traffic": FWD_GEMM_DRAM_BYTES_PER_LAUNCH,
                 "peak_kind": f"bf16 dense, sustained ({pk['source']})",
                 "frac_of_burst_peak": achieved / tc_burst,
                 "per_launch_ms": gemm_ms,
