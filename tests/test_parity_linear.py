@@ -59,6 +59,8 @@ def _layer(q, N, K, M, r, alpha, seed, dq=True, wdtype="bf16"):
     (384, 512, 257, 32, 8.0, True),
     (256, 640, 513, 64, 16.0, True),
     (136, 256, 700, 128, 64.0, False),
+    (96, 256, 300, 16, 32.0, True),        # N <= 128: the single-SM GEMM engine
+    (128, 192, 257, 8, 16.0, False),
     (512, 1024, 1, 16, 32.0, True),        # decode-sized token counts
     (512, 1024, 4, 16, 32.0, True),
     (512, 1024, 17, 16, 32.0, True),
@@ -164,6 +166,8 @@ def test_forward_mlp_7b_full_size_sampled(q):
     (200, 192, 257, 8, 16.0, True),        # N not a multiple of 64: partial contraction step
     (384, 256, 513, 64, 128.0, False),
     (136, 320, 100, 128, 64.0, True),
+    (512, 128, 300, 16, 32.0, True),       # K <= 128: dX on the single-SM GEMM engine
+    (256, 64, 100, 8, 16.0, False),
     (512, 1024, 1, 16, 32.0, False),       # decode-sized token counts
     (512, 1024, 4, 16, 32.0, True),
 ])
