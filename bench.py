@@ -354,7 +354,9 @@ def run_ours(args, rank, world, local_rank):
                 "peak_kind": f"bf16 dense, sustained ({pk['source']})",
                 "frac_of_burst_peak": achieved / tc_burst,
                 "per_launch_ms": gemm_ms,
-                "algorithmic_flops_per_launch": gemm_flops}
+                "algorithmic_flops_per_launch": gemm_flops,
+                # the same launches counted on the base product 2MNK alone
+                "achieved_base_only": sum(2 * M * N * K for (N, K) in wl.weights) / (sum(gemm_ms) * 1e-3) / 1e12}
 
     # ---- end-to-end through the C ABI with host buffers
     e2e = None
