@@ -182,7 +182,7 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream);
  *   ws device workspace of qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r)
  * Constraints: M >= 1, N % 8 == 0, K % 64 == 0, r in {8,16,32,64,128},
  * alpha finite.  M <= 16 runs the decode (GEMV) kernel, larger M the fused
- * dequantise-in-mainloop tensor-core GEMM.  The decode kernel applies each
+ * dequantise-in-mainloop tensor-core GEMM (on pairs of SMs when N > 128).  The decode kernel applies each
  * block's scale to that block's fp32 partial product (the table rounded to
  * bf16 rather than each scaled weight); the GEMM uses the bf16 weights of
  * nf4_dequantize exactly.  Both are within the layer's tolerance.
