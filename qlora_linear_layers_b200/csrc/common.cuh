@@ -1,6 +1,7 @@
 // Shared device-side helpers for the sm_100a kernels of libqlora_nf4.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -19,6 +20,23 @@ __device__ __forceinline__ void set_status(int* st, int code) {
 }
 
 int* device_status_ptr();   // host: address of the status word on the current device
+
+// Raise a kernel's dynamic shared-memory limit once per device: the attribute
+// belongs to each device's context, so a process driving several GPUs sets it
+// on each.  `done` is the call site's bitmask of devices already set (devices
+// 64 and up are set on every call).
+template <typename K>
+inline void set_smem_attr_once(K kernel, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_relaxed) & bit)) return;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (bit) done.fetch_or(bit, std::memory_order_relaxed);
+}
 
 // Host-side launch accounting (capi.cu): count_launches(n) after every
 // successful group of n kernel launches.

@@ -335,12 +335,8 @@ k_qlora_gemm(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
 template <int MODE, bool DQ>
 static void launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                        const CUtensorMap& d, const GemmArgs& p, int grid, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_qlora_gemm<MODE, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<MODE>());
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr_devs{0};
+  set_smem_attr_once(k_qlora_gemm<MODE, DQ>, (int)smem_bytes<MODE>(), attr_devs);
   k_qlora_gemm<MODE, DQ><<<grid, NUM_THREADS, smem_bytes<MODE>(), s>>>(a, b, c, d, p);
 }
 

@@ -326,12 +326,8 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
 template <int MODE, bool DQ, int BM>
 static cudaError_t launch_pair_bm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
                                   const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(k_qlora_gemm_pair<MODE, DQ, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<MODE, BM>());
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_devs{0};
+  set_smem_attr_once(k_qlora_gemm_pair<MODE, DQ, BM>, (int)smem_bytes<MODE, BM>(), attr_devs);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);

@@ -511,11 +511,8 @@ void launch_gemv_kernel(const CUtensorMap& tw, const CUtensorMap& ta, const CUte
                         const GemvArgs& a, cudaStream_t st) {
   constexpr int smem = (int)sizeof(GemvSmem<NT>) + 1024;
   static_assert(smem + 256 * 32 * 4 <= 232448, "shared memory per CTA");
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_qlora_gemv<DQ, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr_devs{0};
+  set_smem_attr_once(k_qlora_gemv<DQ, NT>, smem, attr_devs);
   k_qlora_gemv<DQ, NT><<<a.P, kThreads, smem, st>>>(tw, ta, tx, a);
 }
 

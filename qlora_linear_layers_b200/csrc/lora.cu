@@ -216,11 +216,8 @@ template <int RP, bool BT>
 static void launch_skinny(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
                           void* Sraw, float* part, cudaStream_t st) {
   constexpr int smem = 3 * (128 * 64 * 2 + RP * 64 * 2);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_lora_skinny<RP, BT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr_devs{0};
+  set_smem_attr_once(k_lora_skinny<RP, BT>, smem, attr_devs);
   const int splits = skinny_splits(M, L);
   const int nkc = (L + 63) / 64;
   const int cps = (nkc + splits - 1) / splits;
