@@ -62,6 +62,16 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     assert lib.qlora_workspace_bytes(_lib.QLORA_OP_DOUBLE_QUANT, 0, 1000, 0, 0) == 2048
+    ws = lambda op, M, N, K, r: lib.qlora_workspace_bytes(op, M, N, K, r)
+    for (N, K, r) in ((18944, 3584, 64), (3584, 18944, 64), (4096, 4096, 16), (200, 192, 8)):
+        fwd = [ws(_lib.QLORA_OP_FWD, M, N, K, r) for M in (1, 4, 16, 17, 300, 8192)]
+        # decode (M <= 16) keeps fp32 partials per token; the GEMM path per token tile
+        assert all(x > 0 for x in fwd)
+        assert fwd[0] <= fwd[1] <= fwd[2] and fwd[3] <= fwd[4] <= fwd[5]
+        assert fwd[2] >= 16 * (N + r) * 4                      # one fp32 partial per output
+        # the backward holds the transposed dequantised weight deq(W)^T in bf16
+        for M in (17, 300, 8192):
+            assert ws(_lib.QLORA_OP_BWD, M, N, K, r) >= 2 * N * K
 
 
 def test_validation_before_any_device_call(lib):
