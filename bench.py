@@ -44,11 +44,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA NF4 linear TFLOP/s & quant/dequant GB/s, % of B200 roofline"
 # DRAM bytes (read + write) per launch of the fused forward GEMM on this
-# workload, averaged over the step's three launches (gate, up: 364.9 MB each;
-# down: 653.2 MB), from one ncu capture of each shape (dram__bytes_read.sum +
-# dram__bytes_write.sum of `bench.py --case fwd --tokens 8192 --proj 0|2`).
-# The algorithmic bytes are 407 MB per launch.
-FWD_GEMM_DRAM_BYTES_PER_LAUNCH = (2 * 364877568 + 653239040) / 3
+# workload, averaged over the step's three launches, from one ncu capture of
+# each shape (dram__bytes_read.sum + dram__bytes_write.sum of
+# `bench.py --case fwd --tokens 8192 --proj 0|2`).  None until the current
+# kernel has been captured: the figure is reported only for the kernel it
+# was measured on.  The algorithmic bytes are 407 MB per launch.
+FWD_GEMM_DRAM_BYTES_PER_LAUNCH = None
 WORKLOAD = "mlp_7b"
 DECODE_M = 16
 
@@ -61,6 +62,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the per-workload kernel timings after the step")
     ap.add_argument("--case", choices=["fwd", "bwd", "quantize", "dequantize", "dq", "decode"],
                     help="profiling aid: run one operation on one projection and exit")
     ap.add_argument("--proj", type=int, default=0, help="--case: projection 0 gate, 1 up, 2 down")
@@ -342,19 +345,26 @@ def run_ours(args, rank, world, local_rank):
         if "GB/s" in v:
             v["frac_hbm"] = v["GB/s"] / hbm
         else:
-            v["frac_tensor_sustained"] = v["TFLOP/s"] / tc_sus
+            v["frac_tensor"] = v["TFLOP/s"] / tc_burst
     components["per_projection_ms"] = per_proj
 
-    # dominant kernel: the fused NF4-dequant forward GEMM (one launch per projection)
+    # dominant kernel: the fused NF4-dequant forward GEMM (one launch per
+    # projection).  The timed region lasts well under a second, so the burst
+    # peak is the denominator; the sustained peak is reported beside it.
     gemm_flops = [2 * M * N * K + 2 * M * N * r for (N, K) in wl.weights]
     achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     roofline = {"kernel": "k_qlora_gemm_pair<NF4> (fused NF4-dequant forward GEMM + adapter tail, paired SMs)",
-                "bound": "tensor", "achieved": achieved, "peak": tc_sus, "unit": "TFLOP/s",
-                "frac": achieved / tc_sus, "traffic": FWD_GEMM_DRAM_BYTES_PER_LAUNCH,
-                "peak_kind": f"bf16 dense, sustained ({pk['source']})",
-                "frac_of_burst_peak": achieved / tc_burst,
+                "bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": achieved / tc_burst, "traffic": FWD_GEMM_DRAM_BYTES_PER_LAUNCH,
+                "peak_kind": f"bf16 dense, burst ({pk['source']}); the timed region lasts "
+                             f"{total_ms / 1e3:.2f} s",
+                "frac_of_sustained_peak": achieved / tc_sus,
                 "per_launch_ms": gemm_ms,
+                "per_launch_frac": [f / (t * 1e-3) / 1e12 / tc_burst for f, t in zip(gemm_flops, gemm_ms)],
                 "algorithmic_flops_per_launch": gemm_flops,
+                "algorithmic_bytes_per_launch": [N * K // 2 + (N * K // 64) + 4 * ((N * K // 64 + 255) // 256)
+                                                 + 2 * M * K + 2 * M * r + 2 * N * r + 2 * M * N
+                                                 for (N, K) in wl.weights],
                 # the same launches counted on the base product 2MNK alone
                 "achieved_base_only": sum(2 * M * N * K for (N, K) in wl.weights) / (sum(gemm_ms) * 1e-3) / 1e12}
 
@@ -400,6 +410,11 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError("device status set in the end-to-end leg")
 
     clocks = sampler.stop() if sampler else None
+    extras = None
+    if world == 1 and not args.no_extras:
+        del devt, host, ws
+        torch.cuda.empty_cache()
+        extras = workload_timings(q, lib, dev, pk)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(budget_s=20.0)
@@ -420,8 +435,159 @@ def run_ours(args, rank, world, local_rank):
             "e2e": e2e, "gpu_launches": int(launches),
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
             "components": components,
+            "workloads": extras,
         }
         print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Kernel timings on the other workloads (single GPU, after the step)
+# ---------------------------------------------------------------------------
+
+def _time_op(fn, reps, flush):
+    """Median device time (ms) of `fn` over `reps` calls, each preceded by an
+    L2 flush outside the timed events."""
+    import torch
+    stream = torch.cuda.current_stream()
+    fn()                                          # warm-up
+    times = []
+    for _ in range(reps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def workload_timings(q, lib, dev, pk):
+    """Quantise / DQ / dequantise and decode GEMV on the 70B-class projection
+    (28672 x 8192, with and without 1 % outliers, M in {1, 4, 16}); the
+    forward GEMM on the 4096^2 attention projection (4096 tokens, r = 16);
+    the backward on 4096^2 (8192 tokens, r = 64).  Each figure is the median
+    of CUDA-event times of single calls, with L2 flushed (a 256 MB write)
+    before every call."""
+    import torch
+    from qlora_linear_layers_b200 import _lib, synth
+    hbm, tc = pk["hbm_gbs"], pk["bf16_tflops"]
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = lambda: scratch.zero_()
+    gbs = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9
+    out = {"timing": "median of single calls, L2 flushed before each (256 MB write outside the events)",
+           "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc, "source": pk["source"]}}
+
+    # ---- 70B-class projection: bulk quantisation and decode
+    wl = synth.WORKLOADS["decode_70b"]
+    N, K = wl.weights[0]
+    n, na = N * K, N * K // 64
+    r, alpha = wl.r, wl.alpha
+    A = synth.activations(r, K, wl.seed(synth.TID_A), sigma=0.02).to(dev)
+    B = synth.activations(N, r, wl.seed(synth.TID_B), sigma=0.02).to(dev)
+    wsz = max(q.workspace_bytes(_lib.QLORA_OP_FWD, m, N, K, r) for m in wl.decode_M)
+    wsz = max(wsz, q.workspace_bytes(_lib.QLORA_OP_DOUBLE_QUANT, 0, na, 0, 0))
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    dec = {}
+    for outliers in (False, True):
+        W = synth.weight(N, K, wl.seed(synth.TID_W), "bf16", outliers=outliers).to(dev)
+        wq = q.NF4Tensor(
+            packed=torch.empty(n // 2, dtype=torch.uint8, device=dev), rows=N, cols=K,
+            absmax=torch.empty(na, dtype=torch.float32, device=dev),
+            qabsmax=torch.empty(na, dtype=torch.int8, device=dev),
+            dq_scale=torch.empty((na + 255) // 256, dtype=torch.float32, device=dev),
+            dq_mean=torch.empty(4, dtype=torch.float32, device=dev)[:1], double_quant=True)
+        Wd = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        t_q = _time_op(lambda: q.nf4_quantize(W, wq.packed, wq.absmax), 10, flush)
+        t_dq = _time_op(lambda: q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale,
+                                                      wq.dq_mean, ws), 10, flush)
+        t_dd = _time_op(lambda: q.nf4_dequantize(wq, Wd), 10, flush)
+        key = "outliers_1pct" if outliers else "gaussian"
+        rec = {
+            "quantize": {"us": t_q * 1e3, "GB/s": gbs(quant_bytes(n), t_q),
+                         "frac_hbm": gbs(quant_bytes(n), t_q) / hbm, "bytes": quant_bytes(n)},
+            "double_quant": {"us": t_dq * 1e3, "GB/s": gbs(dq_bytes(n), t_dq),
+                             "frac_hbm": gbs(dq_bytes(n), t_dq) / hbm, "bytes": dq_bytes(n)},
+            "quantize_plus_dq": {"us": (t_q + t_dq) * 1e3,
+                                 "GB/s": gbs(quant_bytes(n) + dq_bytes(n), t_q + t_dq),
+                                 "frac_hbm": gbs(quant_bytes(n) + dq_bytes(n), t_q + t_dq) / hbm},
+            "dequantize": {"us": t_dd * 1e3, "GB/s": gbs(dequant_bytes(n), t_dd),
+                           "frac_hbm": gbs(dequant_bytes(n), t_dd) / hbm, "bytes": dequant_bytes(n)},
+        }
+        del W, Wd
+        for m in (wl.decode_M if not outliers else (16,)):
+            X = synth.activations(m, K, wl.seed(synth.TID_X) + m).to(dev)
+            Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
+            t = _time_op(lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, None, ws), 20, flush)
+            nb = decode_bytes(m, N, K, r)
+            rec[f"decode_M{m}"] = {"us": t * 1e3, "GB/s": gbs(nb, t), "frac_hbm": gbs(nb, t) / hbm,
+                                   "bytes": nb}
+        dec[key] = rec
+        del wq
+        torch.cuda.empty_cache()
+    out["decode_70b"] = {"workload": wl.name, **dec}
+    del ws, A, B
+    torch.cuda.empty_cache()
+
+    # ---- the 4096^2 attention projection forward and the 4096^2 backward
+    for name in ("attn_proj_4096", "bwd_4096"):
+        wl = synth.WORKLOADS[name]
+        (N, K), M, r, alpha = wl.weights[0], wl.M, wl.r, wl.alpha
+        W, X, A, B = (t.to(dev) for t in synth.layer_inputs(wl, 0))
+        wq = q.quantize(W)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        T = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(q.workspace_bytes(_lib.QLORA_OP_FWD, M, N, K, r),
+                             q.workspace_bytes(_lib.QLORA_OP_BWD, M, N, K, r)),
+                         dtype=torch.uint8, device=dev)
+        f_fl, b_fl = layer_flops(M, N, K, r)
+        if name == "attn_proj_4096":
+            t = _time_op(lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, T, ws), 10, flush)
+            # the GEMM launch alone, from the library's events around it
+            g = []
+            for _ in range(5):
+                flush()
+                g0, g1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                g0.record(); g1.record()
+                lib.qlora_profile_gemm_events(g0.cuda_event, g1.cuda_event)
+                q.qlora_linear_fwd(wq, X, A, B, alpha, Y, T, ws)
+                g1.synchronize()
+                g.append(g0.elapsed_time(g1))
+            tg = statistics.median(g)
+            gf = 2 * M * N * K + 2 * M * N * r
+            out[name] = {"workload": wl.name,
+                         "fwd": {"us": t * 1e3, "TFLOP/s": f_fl / (t * 1e-3) / 1e12,
+                                 "frac_tensor": f_fl / (t * 1e-3) / 1e12 / tc},
+                         "fwd_gemm_kernel": {"us": tg * 1e3, "TFLOP/s": gf / (tg * 1e-3) / 1e12,
+                                             "frac_tensor": gf / (tg * 1e-3) / 1e12 / tc}}
+        else:
+            dY = synth.upstream_grad(wl, 0).to(dev)
+            dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+            q.qlora_linear_fwd(wq, X, A, B, alpha, Y, T, ws)
+            t = _time_op(lambda: q.qlora_linear_bwd(wq, X, dY, A, B, alpha, dX, dA, dB, T=T, ws=ws),
+                         10, flush)
+            g = []
+            for _ in range(5):
+                flush()
+                g0, g1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                g0.record(); g1.record()
+                lib.qlora_profile_gemm_events(g0.cuda_event, g1.cuda_event)
+                q.qlora_linear_bwd(wq, X, dY, A, B, alpha, dX, dA, dB, T=T, ws=ws)
+                g1.synchronize()
+                g.append(g0.elapsed_time(g1))
+            tg = statistics.median(g)
+            gf = 2 * M * N * K + 2 * M * K * r
+            out[name] = {"workload": wl.name,
+                         "bwd": {"us": t * 1e3, "TFLOP/s": b_fl / (t * 1e-3) / 1e12,
+                                 "frac_tensor": b_fl / (t * 1e-3) / 1e12 / tc},
+                         "bwd_dx_gemm_kernel": {"us": tg * 1e3, "TFLOP/s": gf / (tg * 1e-3) / 1e12,
+                                                "frac_tensor": gf / (tg * 1e-3) / 1e12 / tc}}
+        del W, X, A, B, wq, Y, T, ws
+        torch.cuda.empty_cache()
+    st = q.qlora_check_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the workload timings")
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -583,11 +749,14 @@ def run_case(args):
         raise RuntimeError(f"device status {st}")
 
 
-def main():
-    args = parse()
-    if args.case:
-        run_case(args)
-        return
+def _spawned_rank(local_rank, args, world, port):
+    os.environ.update({"RANK": str(local_rank), "LOCAL_RANK": str(local_rank),
+                       "WORLD_SIZE": str(world), "MASTER_ADDR": "127.0.0.1",
+                       "MASTER_PORT": str(port)})
+    _run(args)
+
+
+def _run(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -599,13 +768,32 @@ def main():
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
     try:
         run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.case:
+        run_case(args)
+        return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not launched by torchrun: start one process per GPU here, ranks
+        # meeting over NCCL on 127.0.0.1
+        import socket
+        import torch.multiprocessing as mp
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        mp.spawn(_spawned_rank, args=(args, args.gpus, port), nprocs=args.gpus, join=True)
+        return
+    _run(args)
 
 
 if __name__ == "__main__":

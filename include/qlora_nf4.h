@@ -25,6 +25,9 @@
  *  - Every device pointer must be 16-byte aligned.
  *  - There is no CPU fallback: without a usable sm_100 device every compute
  *    entry point returns QLORA_ERR_CUDA or QLORA_ERR_UNSUPPORTED.
+ *  - Per-device state (the status word's address, kernel attributes) is set
+ *    up on first use of each device and kept for the life of the process:
+ *    the library must not be used across cudaDeviceReset.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -216,15 +219,24 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY,
  * lives.
  *
  * Same arguments, constraints, results and errors as qlora_linear_fwd, minus
- * ws / ws_bytes.  Scratch is a fixed array of QLORA_FWD_NOALLOC_SCRATCH_BYTES
- * compiled into the library; every GPU that loads the library holds it until
- * the process exits.  Calls whose qlora_workspace_bytes(QLORA_OP_FWD, M, N, K,
- * r) exceeds that size return QLORA_ERR_WORKSPACE before anything is enqueued
- * (8192 tokens at r = 64 need about 11 MiB; with r <= 64 the limit is
- * about 260,000 tokens, with r = 128 about 26,000).
+ * ws / ws_bytes; the argument checks run first and in the same order.
+ * Scratch is a fixed array of QLORA_FWD_NOALLOC_SCRATCH_BYTES compiled into
+ * the library; every GPU that loads the library holds it until the process
+ * exits.  A call whose qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r) exceeds
+ * that size returns QLORA_ERR_WORKSPACE before anything is enqueued.  That
+ * size depends on M, N, K and r together and is not monotonic in M (the
+ * split-contraction partial sums of X A^T vanish once M alone fills the GPU;
+ * the decode path's partials grow with N), so no single token limit exists:
+ * check qlora_workspace_bytes(QLORA_OP_FWD, M, N, K, r) <=
+ * QLORA_FWD_NOALLOC_SCRATCH_BYTES before relying on this entry point.  For
+ * reference, 8192 tokens at K = 3584, r = 64 need about 11 MiB; with
+ * N = K = 4096 and r = 128 the token counts 18,725-18,816 and 26,215-37,760
+ * are refused while 18,817-26,214 and 37,761 and more are accepted.
  *   - The first call on each device resolves the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and keeps it for the
+ *     life of the process; make that first call before any stream capture,
+ *     and do not use the library across cudaDeviceReset (the kept address,
+ *     like the device status word's, belongs to the context it came from).
  *   - No call allocates or frees memory (no cudaMalloc, cudaFree or
  *     allocating library routine).
  *   - All calls share the array: calls whose work overlaps on the GPU (other

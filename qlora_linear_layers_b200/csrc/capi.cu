@@ -144,6 +144,22 @@ static void take_gemm_events(cudaEvent_t* a, cudaEvent_t* b) {
   g_ev_start = g_ev_stop = nullptr;
 }
 
+// Every check of qlora_linear_fwd's arguments except the workspace, in the
+// order that entry point applies them.
+int validate_fwd_args(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
+                      int r, float alpha, const void* Y, const void* T_save) {
+  int st = check_weight(w);
+  if (st) return st;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!valid_rank(r) || !(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return QLORA_ERR_INVALID_ARG;
+  const int64_t N = w->rows, K = w->cols;
+  if (M < 1 || N % 8 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return QLORA_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
+      (T_save && !aligned16(T_save)))
+    return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
 int* device_status_ptr() {
   DeviceInfo* d = nullptr;
   return current_device(&d) == QLORA_OK ? d->status : nullptr;
@@ -265,15 +281,9 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
 int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
                      int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {
-  int st = check_weight(w);
+  int st = validate_fwd_args(w, X, M, A, B, r, alpha, Y, T_save);
   if (st) return st;
-  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
-  if (!valid_rank(r) || !(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return QLORA_ERR_INVALID_ARG;
   const int64_t N = w->rows, K = w->cols;
-  if (M < 1 || N % 8 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return QLORA_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
-      (T_save && !aligned16(T_save)))
-    return QLORA_ERR_ALIGN;
   const FwdWs lay = fwd_ws(M, N, K, r);
   if (!ws || ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;

@@ -109,7 +109,7 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     mbar_fence_init();
   }
   for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    S.inv127[i] = __fdiv_rn((float)(i - 127), 127.0f);
+    S.inv127[i] = __fdiv_rn((float)(i - 128), 127.0f);   // entry c + 128: any int8 c
   if (warp == 1) {
     tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
     tmem_relinquish_pair();
@@ -241,7 +241,7 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
         }
       } else {
         // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
-        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 127], cur.sg), mu) : cur.a_raw;
+        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 128], cur.sg), mu) : cur.a_raw;
         const Lut l = build_lut(a, p.q);
         const uint32_t wds[8] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w,
                                  cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};

@@ -161,7 +161,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     const int e = i >> 5;
     tbl[i] = pack_bf16x2(p.q[e >> 4], p.q[e & 15]);   // element 2j (high nibble) low half
   }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) S.inv127[i] = __fdiv_rn((float)(i - 127), 127.0f);
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) S.inv127[i] = __fdiv_rn((float)(i - 128), 127.0f);   // entry c + 128: any int8 c
   if (threadIdx.x == 0) {
     S.abort = 0;
     for (int i = 0; i < kStages; ++i) {
@@ -354,7 +354,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[s]);
         // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
-        const float a_mine = DQ ? __fadd_rn(__fmul_rn(S.inv127[qs + 127], fs), mu) : fs;
+        const float a_mine = DQ ? __fadd_rn(__fmul_rn(S.inv127[qs + 128], fs), mu) : fs;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const float ag = __shfl_sync(0xffffffffu, a_mine, g * 4 + t);

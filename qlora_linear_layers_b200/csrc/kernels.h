@@ -18,4 +18,8 @@ int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, floa
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms);
 
+// All argument checks of qlora_linear_fwd except the workspace (capi.cu).
+int validate_fwd_args(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
+                      int r, float alpha, const void* Y, const void* T_save);
+
 }  // namespace qnf4

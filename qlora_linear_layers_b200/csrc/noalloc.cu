@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/qlora_nf4.h"
+#include "kernels.h"
 
 namespace {
 
@@ -56,11 +57,14 @@ int scratch_for_current_device(void** out) {
 extern "C" int qlora_linear_fwd_noalloc(const nf4_weight* w, const void* X, int64_t M,
                                         const void* A, const void* B, int r, float alpha,
                                         void* Y, void* T_save, qlora_stream_t stream) {
-  if (!w) return QLORA_ERR_INVALID_ARG;
+  // the same argument checks, in the same order, as qlora_linear_fwd; only
+  // then the size of the fixed scratch
+  int st = qnf4::validate_fwd_args(w, X, M, A, B, r, alpha, Y, T_save);
+  if (st) return st;
   const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, M, w->rows, w->cols, r);
   if (need > kScratchBytes) return QLORA_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const int st = scratch_for_current_device(&scratch);
+  st = scratch_for_current_device(&scratch);
   if (st) return st;
   return qlora_linear_fwd(w, X, M, A, B, r, alpha, Y, T_save, scratch, kScratchBytes, stream);
 }

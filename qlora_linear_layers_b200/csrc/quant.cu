@@ -403,7 +403,7 @@ k_nf4_dequantize(const uint8_t* __restrict__ packed, int64_t nchunks,
   __shared__ float s_q[16];
   __shared__ float s_inv127[256];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
-  s_inv127[threadIdx.x] = __fdiv_rn((float)((int)threadIdx.x - 127), 127.0f);
+  s_inv127[threadIdx.x] = __fdiv_rn((float)((int)threadIdx.x - 128), 127.0f);   // entry c + 128: any int8 c
   __syncthreads();
   const float mu = DQ ? dq_mean[0] : 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -411,7 +411,7 @@ k_nf4_dequantize(const uint8_t* __restrict__ packed, int64_t nchunks,
        chunk += stride) {
     const int64_t blk = chunk >> 3;
     float a;
-    if (DQ) a = __fadd_rn(__fmul_rn(s_inv127[qabsmax[blk] + 127], __ldg(dq_scale + (blk >> 8))), mu);
+    if (DQ) a = __fadd_rn(__fmul_rn(s_inv127[qabsmax[blk] + 128], __ldg(dq_scale + (blk >> 8))), mu);
     else a = __ldg(absmax + blk);
     const uint32_t wd = __ldcs(reinterpret_cast<const uint32_t*>(packed) + chunk);
     uint32_t o[4];

@@ -304,6 +304,149 @@ def test_double_quantize_constant_group():
     assert np.all(oracle.dq_absmax(q, s, mu) == np.float32(0.25))
 
 
+# ---------------------------------------------------------------------------
+# The rounding sequence of double quantisation, restated in exact rationals
+# ---------------------------------------------------------------------------
+
+def _round_binary(x: Fraction, p: int, emin: int) -> Fraction:
+    """Round a rational to the nearest binary float with p significand bits
+    and minimum normal exponent emin (subnormals below), ties to even.
+    Written from the IEEE 754 definition, independent of NumPy."""
+    if x == 0:
+        return Fraction(0)
+    sign = -1 if x < 0 else 1
+    m = abs(x)
+    e = m.numerator.bit_length() - m.denominator.bit_length()
+    if Fraction(2) ** e > m:
+        e -= 1                                   # now 2^e <= m < 2^(e+1)
+    e = max(e, emin)
+    quantum = Fraction(2) ** (e - p + 1)         # spacing of the grid at m
+    k, rem = divmod(m, quantum)                  # m = k * quantum + rem
+    half = quantum / 2
+    if rem > half or (rem == half and k % 2 == 1):
+        k += 1
+    return sign * k * quantum
+
+
+def _rn32(x: Fraction) -> Fraction:
+    return _round_binary(x, 24, -126)
+
+
+def _rn64(x: Fraction) -> Fraction:
+    return _round_binary(x, 53, -1022)
+
+
+def _round_half_even_int(x: Fraction) -> int:
+    k = math.floor(x)
+    rem = x - k
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    return k
+
+
+def _dq_exact(a: np.ndarray, group: int = 256):
+    """Double quantisation restated step by step in rationals: the mean
+    RN32(RN64(exact sum)/n) with the fp64 division correctly rounded, then per
+    group d = RN32(a - mu), s_g = max|d|, t = RN32(d / s_g), u = RN32(t * 127),
+    c = round-half-even(u) (page "QLoRA Explained", section "Shrink the scale
+    factors too"; the int8 scale-and-round reading of the same page)."""
+    fa = [Fraction(float(v)) for v in a]
+    total = _rn64(sum(fa, Fraction(0)))
+    mu = _rn32(_rn64(total / len(fa)))
+    d = [_rn32(v - mu) for v in fa]
+    codes, scales = [], []
+    for g0 in range(0, len(d), group):
+        dg = d[g0:g0 + group]
+        sg = max(abs(v) for v in dg)
+        scales.append(sg)
+        for v in dg:
+            if sg == 0:
+                codes.append(0)
+                continue
+            t = _rn32(v / sg)
+            u = _rn32(t * 127)
+            codes.append(max(-127, min(127, _round_half_even_int(u))))
+    return codes, scales, mu
+
+
+def _tie_offsets(sg: float, count: int):
+    """Offsets e (exact fp32, |e| < sg) for which RN32(RN32(e / sg) * 127) is
+    exactly k + 1/2: the integer step then meets a tie."""
+    out = []
+    fsg = Fraction(sg)
+    for k in range(126, -1, -1):
+        target = Fraction(2 * k + 1, 2 * 127) * fsg
+        e0 = np.float32(float(target))
+        for step in range(-24, 25):
+            e = np.float32(e0)
+            for _ in range(abs(step)):
+                e = np.nextafter(e, np.float32(np.inf if step > 0 else -np.inf))
+            t = _rn32(Fraction(float(e)) / fsg)
+            if _rn32(t * 127) == Fraction(2 * k + 1, 2):
+                out.append(float(e))
+                break
+        if len(out) >= count:
+            break
+    return out
+
+
+def test_double_quantize_rounding_sequence_exact_rationals():
+    """Every code, scale and the mean of oracle.double_quantize equal the
+    rational restatement of the reading c = rint(RN32(RN32(d / s_g) * 127)),
+    rounding each step to fp32 by hand.  The inputs include constructed
+    near-ties of the integer step (u = k + 1/2 exactly), where swapping the
+    order to RN32(d * 127) / s_g or rounding half away from zero changes
+    the code."""
+    rng = np.random.default_rng(31)
+    # (1) random Gaussian-like absmax values: 2 full groups + a partial one
+    a1 = (np.abs(rng.standard_normal(600)) * 0.02 + 0.01).astype(np.float32)
+    # (2) exact ties: a = 1 +/- e in symmetric pairs, so the mean is exactly 1,
+    # d = +/-e exactly, and s_g = 0.5 (the group holds 1.5 and 0.5)
+    ties = _tie_offsets(0.5, 100)
+    assert len(ties) >= 40
+    a2 = [1.5, 0.5]
+    for e in ties:
+        a2 += [1.0 + e, 1.0 - e]
+    a2 = np.array(a2[:256], dtype=np.float32)
+    assert np.all((a2.astype(np.float64) - 1.0) == np.array([Fraction(float(v)) - 1 for v in a2], dtype=np.float64))
+    for a in (a1, a2):
+        q, s, mu = oracle.double_quantize(a)
+        codes, scales, mu_x = _dq_exact(a)
+        assert Fraction(float(mu)) == mu_x
+        assert [Fraction(float(v)) for v in s] == scales
+        assert q.astype(int).tolist() == codes
+    # the ties decide: rounding half away from zero changes those codes
+    q2, _, mu2 = oracle.double_quantize(a2)
+    assert mu2 == np.float32(1.0)
+    away = 0
+    for v, c in zip(a2, q2.astype(int)):
+        u = _rn32(_rn32((Fraction(float(v)) - 1) / Fraction(0.5)) * 127)
+        if u - math.floor(u) == Fraction(1, 2):
+            away += int(math.copysign(math.floor(abs(u)) + 1, float(u))) != c
+    assert away >= 20
+    # (3) the order of the two fp32 steps matters: with s_g not a power of
+    # two, offsets near a tie give other codes under RN32(RN32(d * 127) / s_g)
+    sg = float(np.float32(round(0.37 * 2 ** 23) / 2 ** 23))
+    fsg = Fraction(sg)
+    a3, n_swap = [1.0 + sg, 1.0 - sg], 0
+    for k in range(1, 127):
+        e0 = round(float(Fraction(2 * k + 1, 254) * fsg) * 2 ** 23)
+        for j in range(e0 - 200, e0 + 201):
+            d = Fraction(j, 2 ** 23)
+            ours = _round_half_even_int(_rn32(_rn32(d / fsg) * 127))
+            other = _round_half_even_int(_rn32(_rn32(d * 127) / fsg))
+            if ours != other:
+                a3 += [1.0 + float(d), 1.0 - float(d)]
+                n_swap += 1
+                break
+    assert n_swap >= 5
+    a3 = np.array(a3[:256], dtype=np.float32)
+    q3, s3, mu3 = oracle.double_quantize(a3)
+    codes, scales, mu_x = _dq_exact(a3)
+    assert mu3 == np.float32(1.0) and s3[0] == np.float32(sg)
+    assert q3.astype(int).tolist() == codes
+
+
 def test_storage_closed_forms(golden):
     g = golden
     n = 4096 * 4096

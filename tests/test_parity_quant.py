@@ -3,9 +3,9 @@
 All results must be bit-exact: packed codes, fp32 absmax, int8 qabsmax, fp32
 group scales, the fp32 mean and the dequantised bf16 weights.  Small
 workloads are compared in full; the full-size weights are quantised whole on
-the GPU and compared on sampled blocks (quantise and dequantise are local to
-a block) and in full for the double quantisation (the oracle handles a few
-million scales in seconds).
+the GPU and their absmax and double quantisation compared in full against the
+oracle's own (computed from the weight), the codes and dequantised weights on
+sampled blocks (quantise and dequantise are local to a block).
 """
 
 import numpy as np
@@ -105,27 +105,31 @@ def test_nonfinite_sets_status(q):
 
 
 def _sampled(q, W_cpu, nsample=96, seed=0):
-    """Quantise the whole matrix on the GPU; compare sampled blocks, and the
-    double quantisation in full."""
+    """Quantise the whole matrix on the GPU.  The oracle computes every block
+    absmax and the double quantisation of the whole tensor from the weight
+    itself (never from a GPU output); both are compared in full, the codes
+    and dequantised weights on sampled blocks (they are local to a block)."""
     wq = q.quantize(W_cpu.cuda(), double_quant=True)
     Wdeq = q.dequantize(wq)
     assert q.qlora_check_status() == 0
-    nblk = wq.absmax.numel()
-    rng = np.random.default_rng(seed)
-    blocks = np.unique(np.concatenate([rng.choice(nblk, nsample, replace=False), [0, nblk - 1]]))
-    Wflat = W_cpu.reshape(-1, 64)
+    Wnp = W_cpu.float().numpy()
+    a = oracle.block_absmax(Wnp)
     absmax = _np(wq.absmax)
-    qa, s, mu = oracle.double_quantize(absmax)
+    assert np.array_equal(absmax.view(np.uint32), a.view(np.uint32))
+    qa, s, mu = oracle.double_quantize(a)
     assert np.array_equal(_np(wq.qabsmax), qa)
     assert np.array_equal(_np(wq.dq_scale).view(np.uint32), s.view(np.uint32))
-    assert _np(wq.dq_mean)[0] == np.float32(mu)
+    assert _np(wq.dq_mean)[0].view(np.uint32) == np.float32(mu).view(np.uint32)
     ah = oracle.dq_absmax(qa, s, mu)
+    nblk = a.size
+    rng = np.random.default_rng(seed)
+    blocks = np.unique(np.concatenate([rng.choice(nblk, nsample, replace=False), [0, nblk - 1]]))
+    Wflat = Wnp.reshape(-1, 64)
     packed = _np(wq.packed).reshape(-1, 32)
     deq = Wdeq.reshape(-1, 64)
     for b in blocks:
-        wb = Wflat[b:b + 1].float().numpy()
-        codes, a = oracle.quantize(wb)
-        assert absmax[b].view(np.uint32) == a[0].view(np.uint32)
+        codes, ab = oracle.quantize(Wflat[b:b + 1])
+        assert ab[0].view(np.uint32) == a[b].view(np.uint32)
         assert np.array_equal(packed[b], oracle.pack(codes))
         ref = oracle.dequantize(oracle.pack(codes), ah[b:b + 1], (1, 64))
         assert np.array_equal(deq[b].float().cpu().numpy().view(np.uint32),
