@@ -7,7 +7,10 @@ One step is one pass of the whole hot path over one batch of the 7B-class
 decoder MLP workload (gate/up W 18944x3584, down W 3584x18944, 8192 tokens,
 r=64, alpha=16), for each of the three projections:
 
-    nf4_quantize + nf4_double_quantize   (quantise the frozen bf16 weight)
+    qlora_quantize_4bit + nf4_double_quantize_hist
+                                         (quantise the frozen bf16 weight; the
+                                          DQ mean's histogram is built while
+                                          quantising)
     nf4_dequantize                       (bf16 export of the base weight)
     qlora_linear_fwd                     (fused NF4-dequant GEMM + adapter)
     qlora_linear_bwd                     (dX, dA, dB; T saved by the forward)
@@ -98,7 +101,12 @@ def quant_bytes(n):          # read bf16, write codes + fp32 absmax
     return n * 2 + n // 2 + 4 * (n // 64)
 
 
-def dq_bytes(n):             # read absmax twice (sum, codes), write int8 + group scales
+def dq_bytes(n):             # finalise pass: read absmax, write int8 + group scales
+    na = n // 64                 # (the quantise pass built the mean's histogram)
+    return 4 * na + na + 4 * ((na + 255) // 256)
+
+
+def dq_standalone_bytes(n):  # from an absmax array: read it twice (histogram, codes)
     na = n // 64
     return 8 * na + na + 4 * ((na + 255) // 256)
 
@@ -228,6 +236,7 @@ def run_ours(args, rank, world, local_rank):
                        q.workspace_bytes(_lib.QLORA_OP_FWD, DECODE_M, N, K, r),
                        q.workspace_bytes(_lib.QLORA_OP_DOUBLE_QUANT, 0, N * K // 64, 0, 0))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    hist = torch.empty(256, dtype=torch.int64, device=dev)
     torch.cuda.synchronize()
 
     comps = ("quantize", "double_quant", "dequantize", "fwd", "bwd", "decode")
@@ -237,9 +246,11 @@ def run_ours(args, rank, world, local_rank):
         wq = d["wq"]
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if record is not None else None
         if ev: ev[0].record(stream)
-        q.nf4_quantize(d["W"], wq.packed, wq.absmax)
+        # quantise, building the DQ mean's histogram on the way; then the DQ pass
+        q.qlora_quantize_4bit(d["W"], wq.packed, wq.absmax, 0, hist)
         if ev: ev[1].record(stream)
-        q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws)
+        q.nf4_double_quantize_hist(wq.absmax, hist, wq.absmax.numel(), wq.qabsmax, wq.dq_scale,
+                                   wq.dq_mean)
         if ev: ev[2].record(stream)
         q.nf4_dequantize(wq, d["Wdeq"])
         if ev: ev[3].record(stream)
@@ -498,16 +509,23 @@ def workload_timings(q, lib, dev, pk):
             dq_scale=torch.empty((na + 255) // 256, dtype=torch.float32, device=dev),
             dq_mean=torch.empty(4, dtype=torch.float32, device=dev)[:1], double_quant=True)
         Wd = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
-        t_q = _time_op(lambda: q.nf4_quantize(W, wq.packed, wq.absmax), 10, flush)
-        t_dq = _time_op(lambda: q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale,
-                                                      wq.dq_mean, ws), 10, flush)
+        hist = torch.empty(256, dtype=torch.int64, device=dev)
+        t_q = _time_op(lambda: q.qlora_quantize_4bit(W, wq.packed, wq.absmax, 0, hist), 10, flush)
+        t_dq = _time_op(lambda: q.nf4_double_quantize_hist(wq.absmax, hist, na, wq.qabsmax,
+                                                           wq.dq_scale, wq.dq_mean), 10, flush)
+        t_dqs = _time_op(lambda: q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale,
+                                                       wq.dq_mean, ws), 10, flush)
         t_dd = _time_op(lambda: q.nf4_dequantize(wq, Wd), 10, flush)
         key = "outliers_1pct" if outliers else "gaussian"
         rec = {
             "quantize": {"us": t_q * 1e3, "GB/s": gbs(quant_bytes(n), t_q),
                          "frac_hbm": gbs(quant_bytes(n), t_q) / hbm, "bytes": quant_bytes(n)},
             "double_quant": {"us": t_dq * 1e3, "GB/s": gbs(dq_bytes(n), t_dq),
-                             "frac_hbm": gbs(dq_bytes(n), t_dq) / hbm, "bytes": dq_bytes(n)},
+                             "frac_hbm": gbs(dq_bytes(n), t_dq) / hbm, "bytes": dq_bytes(n),
+                             "pass": "finalise from the histogram built while quantising"},
+            "double_quant_standalone": {"us": t_dqs * 1e3, "GB/s": gbs(dq_standalone_bytes(n), t_dqs),
+                                        "frac_hbm": gbs(dq_standalone_bytes(n), t_dqs) / hbm,
+                                        "bytes": dq_standalone_bytes(n)},
             "quantize_plus_dq": {"us": (t_q + t_dq) * 1e3,
                                  "GB/s": gbs(quant_bytes(n) + dq_bytes(n), t_q + t_dq),
                                  "frac_hbm": gbs(quant_bytes(n) + dq_bytes(n), t_q + t_dq) / hbm},
@@ -724,12 +742,14 @@ def run_case(args):
                          q.workspace_bytes(_lib.QLORA_OP_BWD, M, N, K, r), 2048),
                      dtype=torch.uint8, device=dev)
     dX, dA, dB = torch.empty_like(X), torch.empty_like(A), torch.empty_like(B)
+    hist = torch.empty(256, dtype=torch.int64, device=dev)
     ops = {
         "fwd": lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, T, ws),
         "decode": lambda: q.qlora_linear_fwd(wq, X, A, B, alpha, Y, None, ws),
         "bwd": lambda: q.qlora_linear_bwd(wq, X, dY, A, B, alpha, dX, dA, dB, T=T, ws=ws),
-        "quantize": lambda: q.nf4_quantize(W, wq.packed, wq.absmax),
-        "dq": lambda: q.nf4_double_quantize(wq.absmax, wq.qabsmax, wq.dq_scale, wq.dq_mean, ws),
+        "quantize": lambda: q.qlora_quantize_4bit(W, wq.packed, wq.absmax, 0, hist),
+        "dq": lambda: q.nf4_double_quantize_hist(wq.absmax, hist, wq.absmax.numel(), wq.qabsmax,
+                                                 wq.dq_scale, wq.dq_mean),
         "dequantize": lambda: q.nf4_dequantize(wq, Wd),
     }
     torch.cuda.synchronize()

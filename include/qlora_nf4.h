@@ -56,6 +56,24 @@ typedef enum {
 
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
+/* 4-bit data types ([QE] config walk-through: bnb_4bit_quant_type picks the
+ * table; "the library's other 4-bit option is a small floating-point layout
+ * ... it costs exactly the same memory").
+ *   QLORA_QUANT_NF4: the 16 normal quantiles of [QE] "That is NF4"; code =
+ *     rank of the value (0 = -1, 7 = exact 0, 15 = +1).
+ *   QLORA_QUANT_FP4: a 4-bit float, sign bit 3, 2 exponent bits, 1 mantissa
+ *     bit, no infinities or NaNs: code c holds
+ *     (-1)^(c>>3) * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[c & 7] / 6, so that the
+ *     largest magnitude meets the block absmax.  Code 8 (-0) decodes to -0
+ *     and is never produced by quantisation. */
+typedef enum { QLORA_QUANT_NF4 = 0, QLORA_QUANT_FP4 = 1 } qlora_quant_type;
+
+/* Bytes of the double-quantisation exponent histogram: 256 int64 bins; bin e
+ * holds the sum of the 24-bit significands of the absmax values whose fp32
+ * exponent field is e (bin 255 unused).  Histograms of disjoint parts of a
+ * tensor add up (integer sum) to the whole tensor's histogram. */
+#define QLORA_DQ_HIST_BYTES 2048
+
 /* Operation ids for qlora_workspace_bytes(). */
 typedef enum {
   QLORA_OP_DOUBLE_QUANT = 0,
@@ -79,10 +97,12 @@ typedef enum {
  *   dq_scale [ceil(rows*cols/64/256)] fp32 group scales (double_quant == 1)
  *   dq_mean  [1] fp32 per-tensor mean offset, device     (double_quant == 1)
  *
- * Dequantised value of element i in block b (code c, table q):
+ * Dequantised value of element i in block b (code c, table q of quant_type):
  *   a^ = absmax[b]                                              (no DQ)
  *   a^ = RN32(RN32(RN32(qabsmax[b]/127) * dq_scale[b/256]) + dq_mean) (DQ)
  *   w' = RNbf16(RN32(q[c] * a^))
+ * quant_type is QLORA_QUANT_NF4 (0) or QLORA_QUANT_FP4 (1); a zero-filled
+ * struct is NF4.
  */
 typedef struct {
   const uint8_t* packed;
@@ -95,6 +115,7 @@ typedef struct {
   const float* dq_scale;
   const float* dq_mean;
   int32_t dq_blocksize;   /* must be 256 */
+  int32_t quant_type;     /* QLORA_QUANT_NF4 or QLORA_QUANT_FP4 */
 } nf4_weight;
 
 /* ---- host-only queries (no GPU needed) -------------------------------- */
@@ -106,6 +127,13 @@ typedef struct {
  * Writes 16 (resp. 15) floats.  Returns QLORA_OK or QLORA_ERR_INVALID_ARG. */
 int nf4_code_table(float* table16);
 int nf4_code_thresholds(float* thresholds15);
+
+/* The same for either 4-bit type: table16 receives the value of each code;
+ * thresholds15 the decision thresholds between consecutive distinct values,
+ * ascending (15 for NF4, 14 for FP4), and *count their number.  Returns
+ * QLORA_OK or QLORA_ERR_INVALID_ARG. */
+int qlora_code_table(int quant_type, float* table16);
+int qlora_code_thresholds(int quant_type, float* thresholds15, int* count);
 
 /* Bytes of caller workspace needed by an operation (0 if none).
  *   QLORA_OP_DOUBLE_QUANT: M, K, r ignored; N = number of absmax values.
@@ -149,6 +177,23 @@ int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols,
                  qlora_stream_t stream);
 
 /*
+ * Blockwise quantisation to either 4-bit type, optionally building the
+ * double-quantisation histogram in the same pass ([QE] "The table, and the
+ * number that stretches it"; "Shrink the scale factors too").  Same as
+ * nf4_quantize with the table of quant_type; ties between two rows go to the
+ * higher value.
+ *   dq_hist  NULL, or device [256] int64 (QLORA_DQ_HIST_BYTES): zeroed by the
+ *            call, then filled with the exponent histogram of this call's
+ *            absmax values (input of nf4_double_quantize_hist).
+ * A shard of a larger weight (a range of whole rows) is quantised the same
+ * way; the shards' histograms summed (for instance by an all-reduce) give
+ * the whole weight's histogram.
+ */
+int qlora_quantize_4bit(const void* W, int dtype, int64_t rows, int64_t cols, int blocksize,
+                        int quant_type, uint8_t* packed, float* absmax, int64_t* dq_hist,
+                        qlora_stream_t stream);
+
+/*
  * Double quantisation of the block scales ([QE] "Shrink the scale factors
  * too").  mean = RN32(RN64(exact sum of absmax) / n) (one per tensor);
  * d = RN32(a - mean); s_g = max|d| over each group of 256 (the last group may
@@ -158,14 +203,28 @@ int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols,
  *   dq_scale device out [ceil(n_absmax/256)] fp32
  *   dq_mean  device out [1] fp32
  *   ws       device workspace of qlora_workspace_bytes(QLORA_OP_DOUBLE_QUANT, ..)
- * The mean is bit-identical for any launch order (exact integer sum).  One
- * cooperative launch (all blocks co-resident, one bounded grid barrier):
- * QLORA_ERR_CUDA if the device refuses it, QLORA_ERR_TIMEOUT in the status
- * word if the barrier gives up.
+ * The mean is bit-identical for any launch order (exact integer sum: an
+ * exponent histogram of the significands, written to ws, then the exact
+ * total rounded once).  A negative, NaN or Inf absmax sets
+ * QLORA_ERR_NONFINITE in the device status word.
  */
 int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
                         int8_t* qabsmax, float* dq_scale, float* dq_mean,
                         void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * The second pass of double quantisation on its own: the mean from a
+ * complete exponent histogram over n_total absmax values (dq_hist from
+ * qlora_quantize_4bit, summed over shards when the weight is sharded), then
+ * the int8 codes and group scales of this array's n_absmax values.  When
+ * sharding, every shard but the last must hold a multiple of 256 absmax
+ * values so that the groups of 256 do not straddle shards; the results then
+ * equal nf4_double_quantize of the whole absmax array bit for bit.
+ *   dq_hist  device [256] int64, read only; n_total >= n_absmax >= 1.
+ */
+int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
+                             int64_t n_total, int dq_blocksize, int8_t* qabsmax,
+                             float* dq_scale, float* dq_mean, qlora_stream_t stream);
 
 /*
  * Dequantise to bf16 ([QE] worked example step 4; "That is NF4": every

@@ -34,6 +34,8 @@ from .nf4 import (  # noqa: F401
     DQ_BLOCKSIZE,
     nf4_table,
     uniform_table,
+    fp4_table,
+    distinct_values,
     thresholds,
     block_absmax,
     normalise,

@@ -80,6 +80,44 @@ def nf4_table() -> np.ndarray:
     return np.array([v / scale for v in levels], dtype=np.float32)
 
 
+def fp4_table() -> np.ndarray:
+    """The FP4 table, by code: a 4-bit float with 1 sign, 2 exponent and 1
+    mantissa bit, scaled so its largest magnitude is 1.
+
+    Page "QLoRA Explained", config walk-through: besides NF4 the library
+    offers "a small floating-point layout" at the same memory cost; section
+    "That is NF4" names the two fields an ordinary float is made of (exponent
+    and mantissa).  Reading: the layout is the E2M1 float (sign bit 3,
+    exponent bits 2-1 with bias 1, mantissa bit 0; no infinities or NaNs):
+
+      e == 0:  value = (-1)^s * m / 2              (subnormal: 0 or 0.5)
+      e >  0:  value = (-1)^s * 2^(e-1) * (1 + m/2)
+
+    giving magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.  Dividing by the largest, 6,
+    maps the table onto [-1, 1] as the absmax scaling needs; RN32 of each
+    quotient.  Code 8 is -0.
+    """
+    vals = []
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        mag = m / 2.0 if e == 0 else 2.0 ** (e - 1) * (1.0 + m / 2.0)
+        vals.append(-(mag / 6.0) if s else mag / 6.0)
+    return np.array(vals, dtype=np.float32)
+
+
+def distinct_values(table: np.ndarray):
+    """The table's distinct values ascending, each with the code that stores
+    it: the lowest code holding the value (+0 rather than -0 for FP4)."""
+    t = np.asarray(table, dtype=np.float32)
+    vals, codes = [], []
+    for c in range(t.size):
+        if not any(float(t[c]) == v for v in vals):
+            vals.append(float(t[c]))
+            codes.append(c)
+    order = np.argsort(vals, kind="stable")
+    return (np.array(vals, dtype=np.float32)[order], np.array(codes, dtype=np.uint8)[order])
+
+
 def thresholds(table: np.ndarray) -> np.ndarray:
     """Decision thresholds for "store the index of the closest row".
 
@@ -90,14 +128,16 @@ def thresholds(table: np.ndarray) -> np.ndarray:
     "The two failures ..." sends 0, exactly between -0.0667 and +0.0667, to
     +0.0667): a value exactly halfway goes to the HIGHER row.
 
-    With ascending rows q_0 < ... < q_15, x is closest-or-tied-up to q_{j+1}
-    rather than q_j exactly when x >= m_j = (q_j + q_{j+1}) / 2.  m_j is exact
-    in fp64 (both q are fp32).  For an fp32 x, x >= m_j  <=>  x >= T_j where
-    T_j is the smallest fp32 that is >= m_j.  Returns the 15 T_j as fp32.
+    With the distinct values ascending, q_0 < ... < q_{v-1}, x is
+    closest-or-tied-up to q_{j+1} rather than q_j exactly when
+    x >= m_j = (q_j + q_{j+1}) / 2.  m_j is exact in fp64 (both q are fp32).
+    For an fp32 x, x >= m_j  <=>  x >= T_j where T_j is the smallest fp32
+    that is >= m_j.  Returns the v - 1 T_j as fp32 (15 for NF4, 14 for FP4,
+    whose +0 and -0 are one value).
     """
-    q = np.asarray(table, dtype=np.float32).astype(np.float64)
-    out = np.empty(15, dtype=np.float32)
-    for j in range(15):
+    q = distinct_values(table)[0].astype(np.float64)
+    out = np.empty(q.size - 1, dtype=np.float32)
+    for j in range(q.size - 1):
         m = (q[j] + q[j + 1]) / 2.0                  # exact in fp64
         t = np.float32(m)                            # RN32(m)
         if float(t) < m:                             # round up if RN went down
@@ -150,13 +190,14 @@ def normalise(W: np.ndarray, absmax: np.ndarray, blocksize: int = BLOCKSIZE) -> 
 
 
 def nearest_code(x: np.ndarray, table: np.ndarray) -> np.ndarray:
-    """Index of the closest table row, ties to the higher row (see thresholds).
-
-    code = #{ j : x >= T_j }.
-    """
+    """Code of the closest table value, ties to the higher value (see
+    thresholds): the k-th smallest distinct value with k = #{ j : x >= T_j },
+    stored under the code distinct_values gives it (for NF4, whose values
+    ascend with the code, code = k)."""
     T = thresholds(table)
+    codes = distinct_values(table)[1]
     x = np.asarray(x, dtype=np.float32)
-    return np.searchsorted(T, x, side="right").astype(np.uint8)
+    return codes[np.searchsorted(T, x, side="right")].astype(np.uint8)
 
 
 def quantize(W: np.ndarray, table: np.ndarray | None = None,

@@ -49,13 +49,14 @@ class NF4Tensor:
     dq_scale: torch.Tensor | None   # fp32 [ceil(n_absmax/256)]
     dq_mean: torch.Tensor | None    # fp32 [1]
     double_quant: bool = True
+    quant_type: int = _lib.QLORA_QUANT_NF4
 
     def c_struct(self) -> _lib.NF4Weight:
         return _lib.NF4Weight(
             packed=_ptr(self.packed), rows=self.rows, cols=self.cols, blocksize=BLOCKSIZE,
             double_quant=1 if self.double_quant else 0,
             absmax=_ptr(self.absmax), qabsmax=_ptr(self.qabsmax), dq_scale=_ptr(self.dq_scale),
-            dq_mean=_ptr(self.dq_mean), dq_blocksize=DQ_BLOCKSIZE)
+            dq_mean=_ptr(self.dq_mean), dq_blocksize=DQ_BLOCKSIZE, quant_type=self.quant_type)
 
     def stored_bytes(self) -> int:
         """Bytes the quantised weight occupies (codes + constants in use)."""
@@ -77,6 +78,35 @@ def nf4_quantize(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Tensor, st
     _lib.check(_lib.load().nf4_quantize(_ptr(W), dt, W.shape[0], W.shape[1], BLOCKSIZE,
                                         _ptr(packed), _ptr(absmax), _stream(stream)),
                "nf4_quantize")
+
+
+def qlora_quantize_4bit(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Tensor,
+                        quant_type: int = _lib.QLORA_QUANT_NF4, dq_hist: torch.Tensor | None = None,
+                        stream=None):
+    """Quantise W (fp32/bf16 [rows, cols]); with dq_hist (int64 [256]) also
+    write the exponent histogram of the block absmax values."""
+    _need_cuda(W, packed, absmax, dq_hist)
+    dt = {torch.float32: _lib.QLORA_F32, torch.bfloat16: _lib.QLORA_BF16}.get(W.dtype)
+    if dt is None:
+        raise ValueError("W must be fp32 or bf16")
+    if dq_hist is not None and (dq_hist.dtype != torch.int64 or dq_hist.numel() != 256):
+        raise ValueError("dq_hist must be int64 [256]")
+    _lib.check(_lib.load().qlora_quantize_4bit(_ptr(W), dt, W.shape[0], W.shape[1], BLOCKSIZE,
+                                               int(quant_type), _ptr(packed), _ptr(absmax),
+                                               _ptr(dq_hist), _stream(stream)),
+               "qlora_quantize_4bit")
+
+
+def nf4_double_quantize_hist(absmax: torch.Tensor, dq_hist: torch.Tensor, n_total: int,
+                             qabsmax: torch.Tensor, dq_scale: torch.Tensor, dq_mean: torch.Tensor,
+                             stream=None):
+    """Second double-quantisation pass from a complete histogram over n_total
+    absmax values (summed over shards when the weight is sharded)."""
+    _need_cuda(absmax, dq_hist, qabsmax, dq_scale, dq_mean)
+    _lib.check(_lib.load().nf4_double_quantize_hist(_ptr(absmax), absmax.numel(), _ptr(dq_hist),
+                                                    int(n_total), DQ_BLOCKSIZE, _ptr(qabsmax),
+                                                    _ptr(dq_scale), _ptr(dq_mean), _stream(stream)),
+               "nf4_double_quantize_hist")
 
 
 def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
@@ -138,37 +168,54 @@ def qlora_check_status(stream=None) -> int:
     return int(_lib.load().qlora_check_status(_stream(stream)))
 
 
-def code_table() -> list[float]:
+def code_table(quant_type: int = _lib.QLORA_QUANT_NF4) -> list[float]:
     buf = (C.c_float * 16)()
-    _lib.check(_lib.load().nf4_code_table(buf), "nf4_code_table")
+    _lib.check(_lib.load().qlora_code_table(int(quant_type), buf), "qlora_code_table")
     return list(buf)
 
 
-def code_thresholds() -> list[float]:
+def code_thresholds(quant_type: int = _lib.QLORA_QUANT_NF4) -> list[float]:
     buf = (C.c_float * 15)()
-    _lib.check(_lib.load().nf4_code_thresholds(buf), "nf4_code_thresholds")
-    return list(buf)
+    cnt = C.c_int(0)
+    _lib.check(_lib.load().qlora_code_thresholds(int(quant_type), buf, C.byref(cnt)),
+               "qlora_code_thresholds")
+    return list(buf)[:cnt.value]
 
 
 # ---------------------------------------------------------------------------
 # Conveniences
 # ---------------------------------------------------------------------------
 
-def quantize(W: torch.Tensor, double_quant: bool = True, stream=None) -> NF4Tensor:
-    rows, cols = W.shape
+def empty_quantized(rows: int, cols: int, device, double_quant: bool = True,
+                    quant_type: int = _lib.QLORA_QUANT_NF4) -> NF4Tensor:
+    """Buffers of a quantised [rows, cols] weight (absmax is kept either way:
+    the quantise pass writes it)."""
     n = rows * cols
-    dev = W.device
-    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
-    absmax = torch.empty(n // BLOCKSIZE, dtype=torch.float32, device=dev)
-    nf4_quantize(W, packed, absmax, stream)
-    q = NF4Tensor(packed, rows, cols, absmax, None, None, None, double_quant)
+    na = n // BLOCKSIZE
+    t = NF4Tensor(torch.empty(n // 2, dtype=torch.uint8, device=device), rows, cols,
+                  torch.empty(na, dtype=torch.float32, device=device), None, None, None,
+                  double_quant, quant_type)
     if double_quant:
-        na = absmax.numel()
-        q.qabsmax = torch.empty(na, dtype=torch.int8, device=dev)
-        q.dq_scale = torch.empty((na + DQ_BLOCKSIZE - 1) // DQ_BLOCKSIZE, dtype=torch.float32,
-                                 device=dev)
-        q.dq_mean = torch.empty(4, dtype=torch.float32, device=dev)[:1]
-        nf4_double_quantize(absmax, q.qabsmax, q.dq_scale, q.dq_mean, stream=stream)
+        t.qabsmax = torch.empty(na, dtype=torch.int8, device=device)
+        t.dq_scale = torch.empty((na + DQ_BLOCKSIZE - 1) // DQ_BLOCKSIZE, dtype=torch.float32,
+                                 device=device)
+        t.dq_mean = torch.empty(4, dtype=torch.float32, device=device)[:1]
+    return t
+
+
+def quantize(W: torch.Tensor, double_quant: bool = True, quant_type: int = _lib.QLORA_QUANT_NF4,
+             stream=None) -> NF4Tensor:
+    """Quantise W; with double quantisation the histogram of the mean is built
+    in the quantise pass and one more pass writes the 8-bit scales."""
+    rows, cols = W.shape
+    q = empty_quantized(rows, cols, W.device, double_quant, quant_type)
+    if not double_quant:
+        qlora_quantize_4bit(W, q.packed, q.absmax, quant_type, None, stream)
+        return q
+    hist = torch.empty(256, dtype=torch.int64, device=W.device)
+    qlora_quantize_4bit(W, q.packed, q.absmax, quant_type, hist, stream)
+    nf4_double_quantize_hist(q.absmax, hist, q.absmax.numel(), q.qabsmax, q.dq_scale, q.dq_mean,
+                             stream)
     return q
 
 

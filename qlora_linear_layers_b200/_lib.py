@@ -26,6 +26,10 @@ QLORA_ERR_WORKSPACE = 8
 QLORA_F32 = 0
 QLORA_BF16 = 1
 
+QLORA_QUANT_NF4 = 0
+QLORA_QUANT_FP4 = 1
+QLORA_DQ_HIST_BYTES = 2048
+
 QLORA_OP_DOUBLE_QUANT = 0
 QLORA_OP_FWD = 1
 QLORA_OP_BWD = 2
@@ -49,6 +53,7 @@ class NF4Weight(C.Structure):
         ("dq_scale", _vp),
         ("dq_mean", _vp),
         ("dq_blocksize", C.c_int32),
+        ("quant_type", C.c_int32),
     ]
 
 
@@ -59,9 +64,13 @@ SIGNATURES = {
     "qlora_status_string": (C.c_char_p, [_i32]),
     "nf4_code_table": (_i32, [C.POINTER(C.c_float)]),
     "nf4_code_thresholds": (_i32, [C.POINTER(C.c_float)]),
+    "qlora_code_table": (_i32, [_i32, C.POINTER(C.c_float)]),
+    "qlora_code_thresholds": (_i32, [_i32, C.POINTER(C.c_float), C.POINTER(C.c_int)]),
     "qlora_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "nf4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "qlora_quantize_4bit": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
     "nf4_double_quantize": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nf4_double_quantize_hist": (_i32, [_vp, _i64, _vp, _i64, _i32, _vp, _vp, _vp, _vp]),
     "nf4_dequantize": (_i32, [C.POINTER(NF4Weight), _vp, _vp]),
     "qlora_linear_fwd": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
                                 _vp, _vp, _vp, _sz, _vp]),

@@ -115,6 +115,7 @@ int launch_status() {
 int check_weight(const nf4_weight* w) {
   if (!w || !w->packed) return QLORA_ERR_INVALID_ARG;
   if (w->blocksize != 64) return QLORA_ERR_UNSUPPORTED;
+  if (w->quant_type != QLORA_QUANT_NF4 && w->quant_type != QLORA_QUANT_FP4) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 64 || w->cols % 64) return QLORA_ERR_SHAPE;
   if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
   if (w->double_quant) {
@@ -171,7 +172,7 @@ using namespace qnf4;
 
 extern "C" {
 
-int qlora_abi_version(void) { return 100; }
+int qlora_abi_version(void) { return 200; }
 
 uint64_t qlora_kernel_launches(void) { return g_launches.load(); }
 
@@ -210,10 +211,26 @@ int nf4_code_thresholds(float* thresholds15) {
   return QLORA_OK;
 }
 
+int qlora_code_table(int quant_type, float* table16) {
+  if (!table16 || (quant_type != QLORA_QUANT_NF4 && quant_type != QLORA_QUANT_FP4))
+    return QLORA_ERR_INVALID_ARG;
+  std::memcpy(table16, host_tables(quant_type).q, 16 * sizeof(float));
+  return QLORA_OK;
+}
+
+int qlora_code_thresholds(int quant_type, float* thresholds15, int* count) {
+  if (!thresholds15 || !count || (quant_type != QLORA_QUANT_NF4 && quant_type != QLORA_QUANT_FP4))
+    return QLORA_ERR_INVALID_ARG;
+  const CodeTables& tb = host_tables(quant_type);
+  std::memcpy(thresholds15, tb.t, (size_t)tb.nt * sizeof(float));
+  *count = tb.nt;
+  return QLORA_OK;
+}
+
 size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   (void)K;
   switch (op) {
-    case QLORA_OP_DOUBLE_QUANT: return 256 * sizeof(unsigned long long);
+    case QLORA_OP_DOUBLE_QUANT: return QLORA_DQ_HIST_BYTES;
     case QLORA_OP_FWD:
       if (M < 1 || N < 1 || !valid_rank(r)) return 0;
       if (K < 1) return 0;
@@ -225,20 +242,31 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   }
 }
 
-int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols, int blocksize,
-                 uint8_t* packed, float* absmax, qlora_stream_t stream) {
+int qlora_quantize_4bit(const void* W, int dtype, int64_t rows, int64_t cols, int blocksize,
+                        int quant_type, uint8_t* packed, float* absmax, int64_t* dq_hist,
+                        qlora_stream_t stream) {
   if (!W || !packed || !absmax) return QLORA_ERR_INVALID_ARG;
   if (dtype != QLORA_F32 && dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
+  if (quant_type != QLORA_QUANT_NF4 && quant_type != QLORA_QUANT_FP4) return QLORA_ERR_INVALID_ARG;
   if (blocksize != 64) return QLORA_ERR_UNSUPPORTED;
-  if (rows < 1 || cols < 64 || cols % 64) return QLORA_ERR_SHAPE;
-  if (!aligned16(W) || !aligned16(packed) || !aligned16(absmax)) return QLORA_ERR_ALIGN;
+  if (rows < 1 || cols < 64 || cols % 64 || rows > ((int64_t)1 << 40) / cols) return QLORA_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(absmax) || (dq_hist && !aligned16(dq_hist)))
+    return QLORA_ERR_ALIGN;
   DeviceInfo* d = nullptr;
   int st = current_device(&d);
   if (st) return st;
-  launch_quantize(W, dtype, rows * cols, packed, absmax, d->status, (cudaStream_t)stream, d->sms);
+  const int n = launch_quantize(W, dtype, rows * cols, quant_type, packed, absmax,
+                                reinterpret_cast<unsigned long long*>(dq_hist), d->status,
+                                (cudaStream_t)stream, d->sms);
   st = launch_status();
-  if (!st) count_launches(1);
+  if (!st) count_launches(n);
   return st;
+}
+
+int nf4_quantize(const void* W, int dtype, int64_t rows, int64_t cols, int blocksize,
+                 uint8_t* packed, float* absmax, qlora_stream_t stream) {
+  return qlora_quantize_4bit(W, dtype, rows, cols, blocksize, QLORA_QUANT_NF4, packed, absmax,
+                             nullptr, stream);
 }
 
 int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize, int8_t* qabsmax,
@@ -259,7 +287,27 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
                                        static_cast<unsigned long long*>(ws), d->status,
                                        (cudaStream_t)stream, d->sms);
   st = launch_status();
-  if (!st && n < 0) st = QLORA_ERR_CUDA;
+  if (!st) count_launches(n);
+  return st;
+}
+
+int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
+                             int64_t n_total, int dq_blocksize, int8_t* qabsmax, float* dq_scale,
+                             float* dq_mean, qlora_stream_t stream) {
+  if (!absmax || !dq_hist || !qabsmax || !dq_scale || !dq_mean) return QLORA_ERR_INVALID_ARG;
+  if (dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
+  if (n_absmax < 1 || n_total < n_absmax || n_total > ((int64_t)1 << 39)) return QLORA_ERR_SHAPE;
+  if (!aligned16(absmax) || !aligned16(dq_hist) || !aligned16(qabsmax) || !aligned16(dq_scale) ||
+      !aligned16(dq_mean))
+    return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  int st = current_device(&d);
+  if (st) return st;
+  const int n = launch_double_quantize_from_hist(absmax, n_absmax,
+                                                 reinterpret_cast<const unsigned long long*>(dq_hist),
+                                                 n_total, qabsmax, dq_scale, dq_mean,
+                                                 (cudaStream_t)stream, d->sms);
+  st = launch_status();
   if (!st) count_launches(n);
   return st;
 }
@@ -297,7 +345,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   if (M <= kDecodeMaxTokens) {
     // decode-sized call: HBM-bound GEMV on the warp-level tensor cores
     const int n = launch_qlora_gemv(w, X, (int)M, A, B, r, scale, Y, T_save,
-                                    reinterpret_cast<float*>(wsb + lay.gemv), host_tables().q,
+                                    reinterpret_cast<float*>(wsb + lay.gemv), host_tables(w->quant_type).q,
                                     d->status, s, d->sms);
     if (n < 0) return QLORA_ERR_CUDA;
     st = launch_status();
@@ -327,7 +375,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   a.na = RP / 64;
   a.double_quant = w->double_quant;
   a.status = d->status;
-  for (int i = 0; i < 16; ++i) a.q[i] = host_tables().q[i];
+  for (int i = 0; i < 16; ++i) a.q[i] = host_tables(w->quant_type).q[i];
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);

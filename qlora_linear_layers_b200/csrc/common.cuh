@@ -42,20 +42,27 @@ inline void set_smem_attr_once(K kernel, int bytes, std::atomic<unsigned long lo
 // successful group of n kernel launches.
 void count_launches(int n);
 
-// The 16 NF4 table values and 15 thresholds, computed on the host and passed
-// to kernels by value (they live in the kernel-parameter constant bank).
-struct Nf4Tables {
-  float q[16];
-  float t[15];
+// A 4-bit data type's tables, computed on the host and passed to kernels by
+// value (they live in the kernel-parameter constant bank).
+struct CodeTables {
+  float q[16];            // value of each code
+  float t[15];            // thresholds between consecutive distinct values, ascending
+  int nt;                 // number of thresholds: 15 (NF4), 14 (FP4)
+  uint8_t rank_code[16];  // code of the k-th smallest distinct value
+  int monotone;           // 1 when code == rank (NF4)
   // Buckets of width 1/16 around the points -1 + b/16: bucket b covers
   // [-1 + (b - 0.5)/16, -1 + (b + 0.5)/16), b = 0..32 (index round(16 x + 16)
   // for x in [-1, 1]); entries 33..63 are unused padding.  At most one
-  // threshold falls in a bucket; code(x) = bucket_base[b] + (x >= bucket_thr[b]).
-  uint8_t bucket_base[64];
+  // threshold falls in a bucket; code(x) = x >= bucket_thr[b] ? bucket_hi[b]
+  // : bucket_lo[b] (thr = 2 where no threshold falls).
   float bucket_thr[64];
+  uint8_t bucket_lo[64];
+  uint8_t bucket_hi[64];
 };
 
-const Nf4Tables& host_tables();   // computed once on the host (table.cpp)
+// Computed once on the host (table.cu); quant_type is QLORA_QUANT_NF4 or
+// QLORA_QUANT_FP4 (anything else: NF4).
+const CodeTables& host_tables(int quant_type = QLORA_QUANT_NF4);
 
 // Every pipeline wait gives up after this much wall time (ns), far above any
 // legitimate wait (the longest stage hand-off is microseconds).

@@ -8,13 +8,24 @@
 
 namespace qnf4 {
 
-void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
-                     int* status, cudaStream_t s, int num_sms);
+// Returns the number of launches (the histogram zeroing counts as one).
+// `hist` (256 u64, or null): zeroed, then filled with the exponent
+// histogram of the block absmax values.
+int launch_quantize(const void* W, int dtype, int64_t n, int quant_type, uint8_t* packed,
+                    float* absmax, unsigned long long* hist, int* status, cudaStream_t s,
+                    int num_sms);
 
-// One cooperative kernel; returns the kernels launched (1), -1 if refused.
+// Double quantisation of an absmax array (histogram + finalise); returns the
+// number of launches.
 int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
-                            float* dq_mean, unsigned long long* hist, int* status,
-                            cudaStream_t s, int num_sms);
+                           float* dq_mean, unsigned long long* hist, int* status, cudaStream_t s,
+                           int num_sms);
+
+// Finalise from a complete histogram over n_total absmax values; returns the
+// number of launches.
+int launch_double_quantize_from_hist(const float* absmax, int64_t n, const unsigned long long* hist,
+                                     int64_t n_total, int8_t* qabsmax, float* dq_scale, float* dq_mean,
+                                     cudaStream_t s, int num_sms);
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms);
 

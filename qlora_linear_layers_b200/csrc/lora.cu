@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(256)
 k_dequant_t(const uint8_t* __restrict__ packed, int N, int K, int dq,
             const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
             const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
-            __nv_bfloat16* __restrict__ Wt, Nf4Tables tb) {
+            __nv_bfloat16* __restrict__ Wt, CodeTables tb) {
   __shared__ uint16_t tile[64][128 + 8];
   __shared__ float s_q[16];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
@@ -478,7 +478,7 @@ void launch_dequant_t(const nf4_weight* w, void* Wt, cudaStream_t st) {
   const dim3 grid((unsigned)((w->cols + 127) / 128), (unsigned)((w->rows + 63) / 64));
   k_dequant_t<<<grid, 256, 0, st>>>(w->packed, (int)w->rows, (int)w->cols, w->double_quant,
                                     w->absmax, w->qabsmax, w->dq_scale, w->dq_mean,
-                                    (__nv_bfloat16*)Wt, host_tables());
+                                    (__nv_bfloat16*)Wt, host_tables(w->quant_type));
 }
 
 // At_pad[k, j] = A[j, k] for j < r, 0 for r <= j < RP.

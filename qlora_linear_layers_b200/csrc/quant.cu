@@ -1,4 +1,5 @@
-// NF4 quantise, double quantise and dequantise kernels (HBM-bound).
+// 4-bit blockwise quantise, double quantise and dequantise kernels
+// (HBM-bound).
 //
 // Page "QLoRA Explained": section "The table, and the number that stretches
 // it" (scale = block absmax, divide, round to the closest row, read back as
@@ -16,26 +17,32 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise: one thread owns one 64-weight block (eight 16-byte bf16 loads or
-// sixteen fp32 ones, a 32-byte code store and its absmax), so the block max,
-// the reciprocal and the stores cost one thread's work per 64 weights.
-// absmax is an integer max over |w| bit patterns (exact; NaN/Inf show up as
-// >= 0x7f800000).
+// Quantise.  Lanes own consecutive 16-byte chunks of the weight, so every
+// warp load instruction reads 512 contiguous bytes; a 64-weight block is 8
+// lanes (bf16) or 16 lanes (fp32), whose absmax is an integer max over |w|
+// bit patterns (exact; NaN/Inf show up as >= 0x7f800000) finished with
+// xor-shuffles inside the lane group.  Each lane issues the loads of four
+// chunks before computing any of them.
 //
 // Code of x = RN32(w / a):  x' = RN32(w * rcp(a)) with the hardware reciprocal
 // (at most 1 ulp off) is within 3.5 ulp of x.  A 64-entry bucket table over
 // [-1, 1] (width 1/16, index = round(16 x + 16), one 8-byte shared load from
 // a copy per lane, so the 32 lanes never meet on a bank) holds the single
-// threshold T that can fall in the bucket and the number of thresholds below
-// it.  When x' is more than 8 ulp from T, x and x'
-// are on the same side of every threshold and the code is base + (x' >= T);
-// a block with any x' within 8 ulp of its T -- or whose absmax is 0 or below
-// 2^-125 -- is redone with the IEEE division (rare; out of line).  Thresholds
-// sit >= 1e-4 from bucket edges (checked on the host), so x' may pick the
-// neighbouring bucket near an edge without effect.
+// threshold T that can fall in the bucket and the codes on either side of
+// it.  When x' is more than 8 ulp from T, x and x' are on the same side of
+// every threshold and the code follows from x' >= T; a lane with any x'
+// within 8 ulp of its T -- or whose block absmax is 0 or below 2^-125 --
+// redoes its own weights with the IEEE division (rare; out of line).
+// Thresholds sit >= 1e-4 from bucket edges (checked on the host), so x' may
+// pick the neighbouring bucket near an edge without effect.
+//
+// With a histogram pointer the kernel also adds every block absmax into the
+// exponent histogram of the double quantisation (below): the significand of
+// each absmax, summed per fp32 exponent, warp-aggregated into shared memory
+// and then into the global 256-bin histogram.
 // ===========================================================================
 
-struct Bucket { float thr; uint32_t base; };
+struct Bucket { float thr; uint32_t codes; };    // codes: lo (NF4), or lo | hi << 8
 
 __device__ __forceinline__ uint32_t bucket_index(float x) {
   // round(16 x + 16) lands in the low mantissa bits of 16 x + 16 + 2^23
@@ -48,138 +55,179 @@ __device__ __forceinline__ float rcp_approx(float a) {
   return r;
 }
 
-// Weight i (0..63) of a block as an fp32 bit pattern, from the block's words.
-template <typename T> struct BlockWords;
-template <> struct BlockWords<__nv_bfloat16> {
-  static constexpr int kWords = 32;               // bf16 pairs, element 2j in the low half
-  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) {
-    return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
+// A 16-byte chunk of the weight.
+template <typename T> struct ChunkT;
+template <> struct ChunkT<__nv_bfloat16> {
+  static constexpr int kE = 8;                   // weights per chunk (bf16 pairs, element 2j low)
+  static constexpr int kL = 8;                   // chunks (lanes) per 64-weight block
+  __device__ __forceinline__ static uint32_t elem(const uint4& v, int i) {
+    const uint32_t w = i < 2 ? v.x : i < 4 ? v.y : i < 6 ? v.z : v.w;
+    return (i & 1) ? (w & 0xFFFF0000u) : (w << 16);
   }
-  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < kWords; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint4& v) {
+    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
     return max(m << 16, m & 0xFFFF0000u);
   }
 };
-template <> struct BlockWords<float> {
-  static constexpr int kWords = 64;
-  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) { return w[i]; }
-  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < kWords; ++j) m = max(m, w[j] & 0x7FFFFFFFu);
-    return m;
+template <> struct ChunkT<float> {
+  static constexpr int kE = 4;
+  static constexpr int kL = 16;
+  __device__ __forceinline__ static uint32_t elem(const uint4& v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+  }
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint4& v) {
+    return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
   }
 };
 
-// Exact codes of block `blk` (x = RN32(w / a), or 0 for a zero block),
-// written straight to `packed`: the rare path, kept out of line so the hot
-// loop keeps its registers.
-template <typename T>
-__device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float a, bool zero_block,
-                                               const Bucket* bks, uint8_t* packed) {
-  uint32_t out[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) out[k] = 0u;
-  for (int i = 0; i < 64; ++i) {
-    float w;
-    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[blk * 64 + i]);
-    else w = reinterpret_cast<const float*>(W)[blk * 64 + i];
-    const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
-    const Bucket bk = bks[bucket_index(x) * 32];
-    const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
-    const int sh = 8 * ((i >> 1) & 3) + ((i & 1) ? 0 : 4);
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k == (i >> 3)) out[k] |= code << sh;
-  }
-  uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
-  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+// Bit position of weight i's code in the lane's packed word: element 2j goes
+// to the high nibble of byte j.
+__device__ __forceinline__ int nib_shift(int i) { return 8 * (i >> 1) + ((i & 1) ? 0 : 4); }
+
+template <bool MONO>
+__device__ __forceinline__ uint32_t code_of(float x, const Bucket* bkl, uint32_t& nearm) {
+  const Bucket b = bkl[bucket_index(x) * 32];
+  // same sign near T, so the bit patterns differ by the ulp distance
+  nearm = min(nearm, (uint32_t)(__float_as_int(x) - __float_as_int(b.thr) + 8));
+  const bool up = x >= b.thr;
+  if (MONO) return b.codes + (up ? 1u : 0u);
+  return up ? (b.codes >> 8) : (b.codes & 0xFFu);
 }
 
-template <typename T>
+// Exact codes of one chunk (x = RN32(w / a), or 0 for a zero block): the
+// rare path, kept out of line so the hot loop keeps its registers.
+template <typename T, bool MONO>
+__device__ __noinline__ uint32_t exact_codes(uint4 v, float a, bool zero_block, const Bucket* bkl) {
+  uint32_t out = 0, unused = 0;
+#pragma unroll
+  for (int i = 0; i < ChunkT<T>::kE; ++i) {
+    const float w = __uint_as_float(ChunkT<T>::elem(v, i));
+    const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
+    out += code_of<MONO>(x, bkl, unused) << nib_shift(i);
+  }
+  return out;
+}
+
+template <typename T, bool MONO, bool HIST>
 __global__ void __launch_bounds__(256)
-k_nf4_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
-               float* __restrict__ absmax, Nf4Tables tb, int* status) {
+k_quantize(const uint4* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ packed,
+           float* __restrict__ absmax, unsigned long long* __restrict__ hist, CodeTables tb,
+           int* status) {
+  using C = ChunkT<T>;
+  constexpr int kU = 4;                          // chunks in flight per lane
   __shared__ Bucket s_bk[64 * 32];               // bucket b, lane l at b * 32 + l
+  __shared__ unsigned long long s_hist[HIST ? 256 : 1];
   for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
     s_bk[i].thr = tb.bucket_thr[i >> 5];
-    s_bk[i].base = tb.bucket_base[i >> 5];
+    s_bk[i].codes = MONO ? tb.bucket_lo[i >> 5]
+                         : (uint32_t)tb.bucket_lo[i >> 5] | ((uint32_t)tb.bucket_hi[i >> 5] << 8);
   }
+  if (HIST)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0ull;
   __syncthreads();
-  const Bucket* bk_lane = s_bk + (threadIdx.x & 31);
-  constexpr int kWords = BlockWords<T>::kWords;
+  const int lane = threadIdx.x & 31;
+  const Bucket* bkl = s_bk + lane;
   bool bad = false;
-  for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblk;
-       blk += (int64_t)gridDim.x * blockDim.x) {
-    uint32_t w[kWords];
-    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * blk;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t base = warp0 * (32 * kU); base < nchunks; base += nwarps * (32 * kU)) {
+    uint4 v[kU];
 #pragma unroll
-    for (int k = 0; k < kWords / 4; ++k) {
-      const uint4 v = __ldg(src + k);
-      w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = base + u * 32 + lane;
+      v[u] = c < nchunks ? __ldcs(W + c) : make_uint4(0u, 0u, 0u, 0u);
     }
-    uint32_t m = BlockWords<T>::absmax_bits(w);
-    if (m >= 0x7F800000u) { bad = true; m = 0; }
-    const float a = __uint_as_float(m);
-    const bool exact_block = m < 0x01000000u;     // a == 0 or a < 2^-125
-    const float inv = exact_block ? 0.0f : rcp_approx(a);
-    uint32_t out[8];
-    uint32_t nearm = 0xFFFFFFFFu;                 // min over the block of (ulp distance to T) + 8
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t o = 0;
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = base + u * 32 + lane;   // a lane group's chunks are all in or all out
+      uint32_t m = C::absmax_bits(v[u]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int i = 8 * k + e;
-        const float x = __fmul_rn(__uint_as_float(BlockWords<T>::elem(w, i)), inv);
-        const Bucket bk = bk_lane[bucket_index(x) * 32];
-        // same sign near T, so the bit patterns differ by the ulp distance
-        nearm = min(nearm, (uint32_t)(__float_as_int(x) - __float_as_int(bk.thr) + 8));
-        const uint32_t code = bk.base + (x >= bk.thr ? 1u : 0u);
-        // element 2j -> high nibble of byte j (fields disjoint: add = or)
-        o += code << (8 * (e >> 1) + ((e & 1) ? 0 : 4));
+      for (int o = 1; o < C::kL; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (m >= 0x7F800000u) { bad = true; m = 0; }
+      const float a = __uint_as_float(m);
+      const bool exact_all = m < 0x01000000u;   // a == 0 or a < 2^-125
+      const float inv = exact_all ? 0.0f : rcp_approx(a);
+      uint32_t nearm = 0xFFFFFFFFu, out = 0;
+#pragma unroll
+      for (int i = 0; i < C::kE; ++i) {
+        const float x = __fmul_rn(__uint_as_float(C::elem(v[u], i)), inv);
+        out += code_of<MONO>(x, bkl, nearm) << nib_shift(i);   // fields disjoint: add = or
       }
-      out[k] = o;
+      if (exact_all || nearm <= 16u) out = exact_codes<T, MONO>(v[u], a, m == 0, bkl);
+      const bool lead = (lane & (C::kL - 1)) == 0;
+      if (c < nchunks) {
+        if (C::kE == 8) reinterpret_cast<uint32_t*>(packed)[c] = out;
+        else reinterpret_cast<uint16_t*>(packed)[c] = (uint16_t)out;
+        if (lead) absmax[c / C::kL] = a;
+      }
+      if (HIST) {
+        const bool add = lead && c < nchunks && m != 0u;
+        const uint32_t e = add ? (m >> 23) : 0xFFFFFFFFu;
+        const uint32_t mant = add ? ((m & 0x7FFFFFu) | (e ? 0x800000u : 0u)) : 0u;
+        const uint32_t grp = __match_any_sync(0xffffffffu, e);
+        const uint32_t sum = __reduce_add_sync(grp, mant);     // at most 4 terms below 2^24
+        if (add && lane == __ffs(grp) - 1) atomicAdd(&s_hist[e], (unsigned long long)sum);
+      }
     }
-    if (exact_block || nearm <= 16u) {
-      exact_block_codes<T>(W, blk, a, m == 0, s_bk, packed);
-    } else {
-      uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
-      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    }
-    absmax[blk] = a;
+  }
+  if (HIST) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 255; i += blockDim.x)
+      if (s_hist[i]) atomicAdd(&hist[i], s_hist[i]);
   }
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
 }
 
-void launch_quantize(const void* W, int dtype, int64_t n, uint8_t* packed, float* absmax,
-                     int* status, cudaStream_t s, int num_sms) {
-  const int64_t nblk = n / 64;
-  const int threads = 256;
-  // one block per thread: other CTAs' loads cover each block's compute
-  int blocks = (int)std::min<int64_t>((nblk + threads - 1) / threads, (int64_t)1 << 30);
-  blocks = std::max(blocks, 1);
-  const Nf4Tables& tb = host_tables();
-  if (dtype == QLORA_BF16)
-    k_nf4_quantize<__nv_bfloat16><<<blocks, threads, 0, s>>>(W, nblk, packed, absmax, tb, status);
+template <typename T, bool MONO>
+static void launch_quantize_t(const void* W, int64_t nchunks, uint8_t* packed, float* absmax,
+                              unsigned long long* hist, const CodeTables& tb, int* status,
+                              cudaStream_t s, int num_sms) {
+  constexpr int kThreads = 256, kPerCta = (kThreads / 32) * 32 * 4;   // chunks per CTA pass
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nchunks + kPerCta - 1) / kPerCta,
+                                                                 (int64_t)num_sms * 4));
+  if (hist)
+    k_quantize<T, MONO, true><<<blocks, kThreads, 0, s>>>((const uint4*)W, nchunks, packed, absmax,
+                                                          hist, tb, status);
   else
-    k_nf4_quantize<float><<<blocks, threads, 0, s>>>(W, nblk, packed, absmax, tb, status);
+    k_quantize<T, MONO, false><<<blocks, kThreads, 0, s>>>((const uint4*)W, nchunks, packed, absmax,
+                                                           nullptr, tb, status);
+}
+
+int launch_quantize(const void* W, int dtype, int64_t n, int quant_type, uint8_t* packed,
+                    float* absmax, unsigned long long* hist, int* status, cudaStream_t s,
+                    int num_sms) {
+  const CodeTables& tb = host_tables(quant_type);
+  int launched = 1;
+  if (hist) {
+    cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
+    ++launched;
+  }
+  const bool bf16 = dtype == QLORA_BF16;
+  const int64_t nchunks = bf16 ? n / 8 : n / 4;
+  if (bf16) {
+    if (tb.monotone) launch_quantize_t<__nv_bfloat16, true>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+    else launch_quantize_t<__nv_bfloat16, false>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+  } else {
+    if (tb.monotone) launch_quantize_t<float, true>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+    else launch_quantize_t<float, false>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+  }
+  return launched;
 }
 
 // ===========================================================================
-// Double quantisation, one cooperative kernel:
-//   1. exact per-tensor sum of absmax: histogram of 24-bit significands per
-//      fp32 exponent (integer adds: exact and order-independent), per block
-//      in shared memory, then added into a global histogram;
-//   2. one grid barrier (counted in bin 255, which no finite value uses);
-//      every block turns the complete histogram into the correctly rounded
-//      fp64 sum and mean = RN32(RN64(sum) / n) -- the same bits everywhere;
-//   3. one warp per group of 256: d = RN32(a - mean), s = max|d|,
-//      c = rint(RN32(RN32(d / s) * 127)) (the group re-read from L2).
+// Double quantisation in two passes.
+//   1. The exact per-tensor sum of absmax as a histogram: the 24-bit
+//      significand of every absmax added (integer adds: exact and
+//      order-independent) into the bin of its fp32 exponent field.  The
+//      quantise kernel builds it on the fly; k_dq_hist builds it from an
+//      absmax array.  Histograms of disjoint parts of a tensor add up to the
+//      tensor's histogram (the multi-GPU sharding sums them).
+//   2. k_dq_finalize: every CTA turns the complete histogram into the
+//      correctly rounded fp64 sum and mean = RN32(RN64(sum) / n) -- the same
+//      bits everywhere -- while its warps load their groups; then one warp
+//      per group of 256: d = RN32(a - mean), s = max|d|,
+//      c = rint(RN32(RN32(d / s) * 127)).
 // ===========================================================================
 
 // Exact integer S = sum_e hist[e] * 2^(max(e,1)-1) in units of 2^-149 (a float
@@ -259,26 +307,17 @@ __device__ float exact_mean_warp(const unsigned long long* hist, int64_t n) {
   return __double2float_rn(__ddiv_rn(S, (double)n));
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
+// Pass 1 on an absmax array (standalone double quantisation).  Every lane of
+// a warp runs the same number of iterations (match/reduce need the full
+// warp); a thread's kU loads are all issued before the first is used.
 __global__ void __launch_bounds__(512)
-k_double_quant(const float* __restrict__ absmax, int64_t n, unsigned long long* __restrict__ hist,
-               int8_t* __restrict__ qabsmax, float* __restrict__ dq_scale, float* __restrict__ mean,
-               int* status) {
+k_dq_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* __restrict__ hist,
+          int* status) {
   __shared__ unsigned long long sh[256];
-  __shared__ float s_mu;
-  __shared__ int s_ok;
   for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0ull;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   bool bad = false;
-  // ---- 1. histogram; every lane of a warp runs the same number of
-  // iterations (match/reduce below need the full warp).  A thread's kU loads
-  // are all issued before the first is used.
   constexpr int kU = 16;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
@@ -312,47 +351,49 @@ k_double_quant(const float* __restrict__ absmax, int64_t n, unsigned long long* 
   for (int i = threadIdx.x; i < 255; i += blockDim.x)
     if (sh[i]) atomicAdd(&hist[i], sh[i]);
   if (bad) set_status(status, QLORA_ERR_NONFINITE);
-  // ---- 2. grid barrier (all blocks are co-resident: cooperative launch),
-  // bounded; then the exact mean from the complete histogram
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    atomicAdd(&hist[255], 1ull);
-    int ok = 1;
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u64(&hist[255]) < (unsigned long long)gridDim.x) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        ok = 0;
-        set_status(status, QLORA_ERR_TIMEOUT);
-        break;
-      }
+}
+
+// Pass 2: the mean over n_total absmax values (this array's n and any other
+// shards' absmax whose histograms were added in), then the int8 codes and
+// fp32 scales of this array's groups.
+__global__ void __launch_bounds__(512)
+k_dq_finalize(const float* __restrict__ absmax, int64_t n, const unsigned long long* __restrict__ hist,
+              int64_t n_total, int8_t* __restrict__ qabsmax, float* __restrict__ dq_scale,
+              float* __restrict__ mean) {
+  __shared__ unsigned long long sh[256];
+  __shared__ float s_mu;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = i < 255 ? __ldcg(&hist[i]) : 0ull;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ngroups = (n + 255) / 256;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  float av[8];
+  auto load = [&](int64_t gg) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t i = gg * 256 + j * 32 + lane;
+      av[j] = i < n ? __ldcg(absmax + i) : 0.0f;
     }
-    s_ok = ok;
-  }
+  };
+  if (g < ngroups) load(g);                      // in flight while the mean is formed
   __syncthreads();
-  if (!s_ok) return;
-  for (int i = threadIdx.x; i < 255; i += blockDim.x) sh[i] = __ldcg(&hist[i]);
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const float mu = exact_mean_warp(sh, n);
-    if (threadIdx.x == 0) {
+  if (warp == 0) {
+    const float mu = exact_mean_warp(sh, n_total);
+    if (lane == 0) {
       s_mu = mu;
       if (blockIdx.x == 0) mean[0] = mu;
     }
   }
   __syncthreads();
-  // ---- 3. one warp per group of 256
   const float mu = s_mu;
-  const int64_t ngroups = (n + 255) / 256;
-  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t g = warp; g < ngroups; g += nwarps) {
+  for (bool first = true; g < ngroups; g += nw, first = false) {
+    if (!first) load(g);
     float d[8];
     float m = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t i = g * 256 + j * 32 + lane;
-      d[j] = (i < n) ? __fsub_rn(__ldcg(absmax + i), mu) : 0.0f;
+      d[j] = (i < n) ? __fsub_rn(av[j], mu) : 0.0f;
       m = fmaxf(m, fabsf(d[j]));
     }
 #pragma unroll
@@ -373,33 +414,40 @@ k_double_quant(const float* __restrict__ absmax, int64_t n, unsigned long long* 
   }
 }
 
-// Returns the number of kernels launched (1), or -1 if the cooperative launch
-// was refused.
+// Returns the number of kernels launched.
+int launch_double_quantize_from_hist(const float* absmax, int64_t n, const unsigned long long* hist,
+                                     int64_t n_total, int8_t* qabsmax, float* dq_scale, float* dq_mean,
+                                     cudaStream_t s, int num_sms) {
+  const int64_t ngroups = (n + 255) / 256;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 15) / 16, (int64_t)num_sms * 2));
+  k_dq_finalize<<<blocks, 512, 0, s>>>(absmax, n, hist, n_total, qabsmax, dq_scale, dq_mean);
+  return 1;
+}
+
 int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, float* dq_scale,
-                           float* dq_mean, unsigned long long* hist, int* status,
-                           cudaStream_t s, int num_sms) {
+                           float* dq_mean, unsigned long long* hist, int* status, cudaStream_t s,
+                           int num_sms) {
   cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
-  // one wide block per SM (fewer blocks meet on the few busy histogram bins)
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 8191) / 8192, (int64_t)num_sms));
-  void* args[] = {(void*)&absmax, (void*)&n, (void*)&hist, (void*)&qabsmax, (void*)&dq_scale,
-                  (void*)&dq_mean, (void*)&status};
-  return cudaLaunchCooperativeKernel((const void*)k_double_quant, dim3(blocks), dim3(512), args, 0, s) ==
-                 cudaSuccess ? 1 : -1;
+  k_dq_hist<<<blocks, 512, 0, s>>>(absmax, n, hist, status);
+  return 2 + launch_double_quantize_from_hist(absmax, n, hist, n, qabsmax, dq_scale, dq_mean, s, num_sms);
 }
 
 // ===========================================================================
-// Dequantise: one thread owns 8 weights (a 4-byte code load, a 16-byte bf16
-// store; contiguous per warp), 8 lanes share a block's scale.
-// w' = RNbf16(RN32(q[code] * a^)), a^ recovered from the double-quantised
-// constants as RN32(RN32(RN32(c / 127) * s_g) + mean).
+// Dequantise: a thread expands 8 weights per chunk (a 4-byte code load, a
+// 16-byte bf16 store; contiguous per warp) and keeps four chunks in flight;
+// 8 lanes share a block's scale.  w' = RNbf16(RN32(q[code] * a^)), a^
+// recovered from the double-quantised constants as
+// RN32(RN32(RN32(c / 127) * s_g) + mean).
 // ===========================================================================
 
 template <bool DQ>
 __global__ void __launch_bounds__(256)
-k_nf4_dequantize(const uint8_t* __restrict__ packed, int64_t nchunks,
-                 const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
-                 const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
-                 uint4* __restrict__ out, Nf4Tables tb) {
+k_dequantize(const uint32_t* __restrict__ packed, int64_t nchunks,
+             const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
+             const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
+             uint4* __restrict__ out, CodeTables tb) {
+  constexpr int kU = 4;
   __shared__ float s_q[16];
   __shared__ float s_inv127[256];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
@@ -407,35 +455,44 @@ k_nf4_dequantize(const uint8_t* __restrict__ packed, int64_t nchunks,
   __syncthreads();
   const float mu = DQ ? dq_mean[0] : 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t chunk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; chunk < nchunks;
-       chunk += stride) {
-    const int64_t blk = chunk >> 3;
-    float a;
-    if (DQ) a = __fadd_rn(__fmul_rn(s_inv127[qabsmax[blk] + 128], __ldg(dq_scale + (blk >> 8))), mu);
-    else a = __ldg(absmax + blk);
-    const uint32_t wd = __ldcs(reinterpret_cast<const uint32_t*>(packed) + chunk);
-    uint32_t o[4];
+  for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c0 < nchunks; c0 += kU * stride) {
+    uint32_t wd[kU];
+    float a[kU];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {            // byte j -> elements 2j (high nibble), 2j+1 (low)
-      const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
-      o[j] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], a), __fmul_rn(s_q[byte & 15], a));
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = c0 + u * stride;
+      const int64_t blk = (c < nchunks ? c : 0) >> 3;
+      wd[u] = c < nchunks ? __ldcs(packed + c) : 0u;
+      if (DQ) a[u] = __fadd_rn(__fmul_rn(s_inv127[qabsmax[blk] + 128], __ldg(dq_scale + (blk >> 8))), mu);
+      else a[u] = __ldg(absmax + blk);
     }
-    __stcs(out + chunk, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t c = c0 + u * stride;
+      if (c >= nchunks) break;
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {            // byte j -> elements 2j (high nibble), 2j+1 (low)
+        const uint32_t byte = (wd[u] >> (8 * j)) & 0xFFu;
+        o[j] = pack_bf16x2(__fmul_rn(s_q[byte >> 4], a[u]), __fmul_rn(s_q[byte & 15], a[u]));
+      }
+      __stcs(out + c, make_uint4(o[0], o[1], o[2], o[3]));
+    }
   }
 }
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms) {
   const int64_t n = w->rows * w->cols;
   const int64_t nchunks = n / 8;
-  int blocks = (int)std::min<int64_t>((nchunks + 255) / 256, (int64_t)num_sms * 8);
+  int blocks = (int)std::min<int64_t>((nchunks + 1023) / 1024, (int64_t)num_sms * 8);
   blocks = std::max(blocks, 1);
-  const Nf4Tables& tb = host_tables();
+  const CodeTables& tb = host_tables(w->quant_type);
   if (w->double_quant)
-    k_nf4_dequantize<true><<<blocks, 256, 0, s>>>(w->packed, nchunks, nullptr, w->qabsmax,
-                                                  w->dq_scale, w->dq_mean, (uint4*)out, tb);
+    k_dequantize<true><<<blocks, 256, 0, s>>>((const uint32_t*)w->packed, nchunks, nullptr, w->qabsmax,
+                                              w->dq_scale, w->dq_mean, (uint4*)out, tb);
   else
-    k_nf4_dequantize<false><<<blocks, 256, 0, s>>>(w->packed, nchunks, w->absmax, nullptr,
-                                                   nullptr, nullptr, (uint4*)out, tb);
+    k_dequantize<false><<<blocks, 256, 0, s>>>((const uint32_t*)w->packed, nchunks, w->absmax, nullptr,
+                                               nullptr, nullptr, (uint4*)out, tb);
 }
 
 }  // namespace qnf4

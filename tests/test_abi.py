@@ -40,7 +40,7 @@ def test_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.SIGNATURES)
-    assert lib.qlora_abi_version() == 100
+    assert lib.qlora_abi_version() == 200
 
 
 def test_library_table_matches_oracle(lib):
@@ -52,6 +52,25 @@ def test_library_table_matches_oracle(lib):
     tb = (C.c_float * 15)()
     assert lib.nf4_code_thresholds(tb) == 0
     assert np.array_equal(np.frombuffer(tb, dtype=np.float32), oracle.thresholds(want))
+
+
+@pytest.mark.parametrize("qt", [_lib.QLORA_QUANT_NF4, _lib.QLORA_QUANT_FP4])
+def test_library_tables_match_oracle_per_type(lib, qt):
+    """The library's tables of both 4-bit types equal the oracle's: values by
+    code and the thresholds between distinct values (FP4: the E2M1 list in
+    the library, the bit-field formula in the oracle)."""
+    buf = (C.c_float * 16)()
+    assert lib.qlora_code_table(qt, buf) == 0
+    got = np.frombuffer(buf, dtype=np.float32)
+    want = oracle.nf4_table() if qt == _lib.QLORA_QUANT_NF4 else oracle.fp4_table()
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    tb = (C.c_float * 15)()
+    cnt = C.c_int(0)
+    assert lib.qlora_code_thresholds(qt, tb, C.byref(cnt)) == 0
+    T = oracle.thresholds(want)
+    assert cnt.value == T.size
+    assert np.array_equal(np.frombuffer(tb, dtype=np.float32)[:cnt.value], T)
+    assert lib.qlora_code_table(7, buf) == _lib.QLORA_ERR_INVALID_ARG
 
 
 def test_status_strings(lib):
@@ -96,3 +115,15 @@ def test_validation_before_any_device_call(lib):
     w.qabsmax = fake
     w.cols = 100
     assert lib.nf4_dequantize(C.byref(w), fake, None) == _lib.QLORA_ERR_SHAPE
+    w.cols = 64
+    w.quant_type = 5
+    assert lib.nf4_dequantize(C.byref(w), fake, None) == _lib.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_4bit(fake, 1, 64, 64, 64, 2, fake, fake, None, None) == \
+        _lib.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_4bit(fake, 1, 64, 64, 64, 1, fake, fake, fake + 8, None) == \
+        _lib.QLORA_ERR_ALIGN
+    # the histogram pass: n_total below the local count, a missing histogram
+    assert lib.nf4_double_quantize_hist(fake, 512, fake, 256, 256, fake, fake, fake, None) == \
+        _lib.QLORA_ERR_SHAPE
+    assert lib.nf4_double_quantize_hist(fake, 512, None, 512, 256, fake, fake, fake, None) == \
+        _lib.QLORA_ERR_INVALID_ARG

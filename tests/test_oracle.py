@@ -80,22 +80,27 @@ def test_nf4_beats_uniform_on_gaussian_weights():
 # ---------------------------------------------------------------------------
 
 def _brute_code(x: float, table) -> int:
-    """argmin_i |x - q_i| in exact rationals; ties -> higher index."""
+    """argmin over codes of |x - q_code| in exact rationals; ties -> the
+    higher value, then the lower code (+0 before -0)."""
     fx = Fraction(float(x))
     best, bi = None, -1
     for i, qi in enumerate(table):
-        d = abs(fx - Fraction(float(qi)))
-        if best is None or d <= best:
-            best, bi = d, i
+        fq = Fraction(float(qi))
+        key = (abs(fx - fq), -fq, i)
+        if best is None or key < best:
+            best, bi = key, i
     return bi
 
 
-@pytest.mark.parametrize("table_name", ["nf4", "uniform"])
+_TABLES = {"nf4": oracle.nf4_table, "uniform": oracle.uniform_table, "fp4": oracle.fp4_table}
+
+
+@pytest.mark.parametrize("table_name", ["nf4", "uniform", "fp4"])
 def test_threshold_code_equals_brute_force(table_name):
-    table = oracle.nf4_table() if table_name == "nf4" else oracle.uniform_table()
+    table = _TABLES[table_name]()
     xs = []
-    q = table.astype(np.float64)
-    for j in range(15):
+    q = np.unique(table.astype(np.float64))
+    for j in range(q.size - 1):
         m = np.float32((q[j] + q[j + 1]) / 2)
         v = m
         for _ in range(5):
@@ -112,17 +117,41 @@ def test_threshold_code_equals_brute_force(table_name):
     assert np.array_equal(got, want)
 
 
-def test_quantize_tiny_blocks_brute_force():
+def test_fp4_table_from_the_float_layout():
+    """The FP4 reading: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 under codes
+    0..7 (the E2M1 values listed, not derived from the bit fields), the sign
+    in bit 3, divided by 6; 15 distinct values ascending with +0 stored as
+    code 0."""
+    t = oracle.fp4_table()
+    listed = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        want = np.float32(listed[c & 7] / 6.0)
+        assert t[c] == (-want if c & 8 else want)
+    assert np.signbit(t[8]) and not np.signbit(t[0])
+    vals, codes = oracle.distinct_values(t)
+    assert vals.size == 15 and np.all(np.diff(vals) > 0)
+    assert vals[0] == -1 and vals[-1] == 1 and codes[7] == 0
+    assert oracle.thresholds(t).size == 14
+    # the ends are exact: the absmax element dequantises to +/- the scale
+    W = np.array([[0.3, -0.02, 0.0, -0.7] + [0.01] * 60], dtype=np.float32)
+    c, a = oracle.quantize(W, t)
+    deq = oracle.dequantize(oracle.pack(c), a, W.shape, table=t)
+    assert deq[0, 3] == oracle.round_bf16(np.float32(-0.7)) and deq[0, 2] == 0.0
+
+
+@pytest.mark.parametrize("table_name", ["nf4", "fp4"])
+def test_quantize_tiny_blocks_brute_force(table_name):
     """Whole quantise path on tiny random blocks vs rational brute force."""
     rng = np.random.default_rng(11)
     W = (rng.standard_normal((4, 128)) * 0.02).astype(np.float32)
-    table = oracle.nf4_table()
+    W[1, :64] = 0.0                                       # zero block: every code is +0's
+    table = _TABLES[table_name]()
     codes, a = oracle.quantize(W, table)
     blk = W.reshape(-1, 64)
     assert np.array_equal(a, np.abs(blk).max(axis=1))
     for b in range(blk.shape[0]):
         for i in range(64):
-            x = np.float32(blk[b, i]) / np.float32(a[b])       # RN32 division
+            x = np.float32(0) if a[b] == 0 else np.float32(blk[b, i]) / np.float32(a[b])   # RN32 division
             assert codes[64 * b + i] == _brute_code(x, table)
 
 

@@ -36,19 +36,20 @@ def rel_err(got, ref):
 
 
 def _oracle_weight(wq, W_cpu):
-    codes, a = oracle.quantize(W_cpu.float().numpy())
+    table = oracle.fp4_table() if wq.quant_type == 1 else oracle.nf4_table()
+    codes, a = oracle.quantize(W_cpu.float().numpy(), table)
     if wq.double_quant:
         qa, s, mu = oracle.double_quantize(a)
         a = oracle.dq_absmax(qa, s, mu)
-    return oracle.dequantize(oracle.pack(codes), a, tuple(W_cpu.shape))
+    return oracle.dequantize(oracle.pack(codes), a, tuple(W_cpu.shape), table=table)
 
 
-def _layer(q, N, K, M, r, alpha, seed, dq=True, wdtype="bf16"):
+def _layer(q, N, K, M, r, alpha, seed, dq=True, wdtype="bf16", qt=0):
     W = synth.weight(N, K, seed + 1, wdtype)
     X = synth.activations(M, K, seed + 2)
     A = synth.activations(r, K, seed + 3, sigma=0.02)
     B = synth.activations(N, r, seed + 4, sigma=0.02)
-    wq = q.quantize(W.cuda(), double_quant=dq)
+    wq = q.quantize(W.cuda(), double_quant=dq, quant_type=qt)
     return W, X, A, B, wq
 
 
@@ -97,11 +98,32 @@ def test_forward_ignores_workspace_contents(q, N, K, M, r, dq):
     assert rel_err(T, Tr) <= TOL
 
 
-def test_forward_identity_is_exact_dequant(q):
+@pytest.mark.parametrize("N,K,M,r,alpha,dq", [
+    (1024, 1024, 16, 8, 16.0, True),
+    (200, 192, 300, 16, 32.0, True),
+    (256, 640, 513, 64, 16.0, False),
+    (96, 256, 300, 16, 32.0, True),
+    (512, 1024, 1, 16, 32.0, True),
+    (512, 1024, 4, 16, 32.0, False),
+])
+def test_forward_small_fp4(q, N, K, M, r, alpha, dq):
+    """The FP4 storage type through the same kernels (the table is the only
+    difference)."""
+    W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=300 * M + r, dq=dq, qt=1)
+    Y, T = q.linear_fwd(wq, X.cuda(), A.cuda(), B.cuda(), alpha)
+    assert q.qlora_check_status() == 0
+    Wd = _oracle_weight(wq, W)
+    Yr, Tr = oracle.linear_fwd(X.float().numpy(), Wd, A.float().numpy(), B.float().numpy(), alpha, r)
+    assert rel_err(Y, Yr) <= TOL
+    assert rel_err(T, Tr) <= TOL
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_forward_identity_is_exact_dequant(q, qt):
     """X = I, A = 0: Y[m, n] = W'[n, m] exactly (one nonzero product per sum)."""
     N, K = 384, 512
     W = synth.weight(N, K, 4242, "bf16")
-    wq = q.quantize(W.cuda(), double_quant=True)
+    wq = q.quantize(W.cuda(), double_quant=True, quant_type=qt)
     X = torch.eye(K, dtype=torch.bfloat16, device="cuda")
     A = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
     B = synth.activations(N, 16, 4243, sigma=0.02).cuda()
@@ -174,6 +196,25 @@ def test_forward_mlp_7b_full_size_sampled(q):
 def test_backward_small(q, N, K, M, r, alpha, pass_T):
     W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=7 * M + r)
     dY = synth.activations(M, N, 7 * M + r + 5)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    _, T = q.linear_fwd(wq, Xc, Ac, Bc, alpha)
+    dX, dA, dB = q.linear_bwd(wq, Xc, dYc, Ac, Bc, alpha, T=T if pass_T else None)
+    assert q.qlora_check_status() == 0
+    Wd = _oracle_weight(wq, W)
+    dXr, dAr, dBr = oracle.linear_bwd(X.float().numpy(), dY.float().numpy(), Wd,
+                                      A.float().numpy(), B.float().numpy(), alpha, r)
+    assert rel_err(dX, dXr) <= TOL
+    assert rel_err(dA, dAr) <= TOL
+    assert rel_err(dB, dBr) <= TOL
+
+
+@pytest.mark.parametrize("N,K,M,r,alpha,pass_T", [
+    (256, 512, 300, 16, 32.0, True),
+    (512, 128, 300, 16, 32.0, False),
+])
+def test_backward_small_fp4(q, N, K, M, r, alpha, pass_T):
+    W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=11 * M + r, qt=1)
+    dY = synth.activations(M, N, 11 * M + r + 5)
     Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
     _, T = q.linear_fwd(wq, Xc, Ac, Bc, alpha)
     dX, dA, dB = q.linear_bwd(wq, Xc, dYc, Ac, Bc, alpha, T=T if pass_T else None)

@@ -31,13 +31,21 @@ def _np(t):
     return t.detach().cpu().numpy()
 
 
-def _check_full(q, W_cpu, double_quant=True):
+NF4, FP4 = 0, 1
+
+
+def _table(qt):
+    return oracle.nf4_table() if qt == NF4 else oracle.fp4_table()
+
+
+def _check_full(q, W_cpu, double_quant=True, qt=NF4):
     Wd = W_cpu.cuda()
-    wq = q.quantize(Wd, double_quant=double_quant)
+    wq = q.quantize(Wd, double_quant=double_quant, quant_type=qt)
     Wdeq = q.dequantize(wq)
     assert q.qlora_check_status() == 0
     Wnp = W_cpu.float().numpy()
-    codes, a = oracle.quantize(Wnp)
+    table = _table(qt)
+    codes, a = oracle.quantize(Wnp, table)
     assert np.array_equal(_np(wq.packed), oracle.pack(codes))
     assert np.array_equal(_np(wq.absmax).view(np.uint32), a.view(np.uint32))
     if double_quant:
@@ -48,23 +56,25 @@ def _check_full(q, W_cpu, double_quant=True):
         ah = oracle.dq_absmax(qa, s, mu)
     else:
         ah = a
-    ref = oracle.dequantize(oracle.pack(codes), ah, Wnp.shape)
+    ref = oracle.dequantize(oracle.pack(codes), ah, Wnp.shape, table=table)
     got = Wdeq.float().cpu().numpy()
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
     return wq
 
 
-def test_tiny_roundtrip_fp32(q):
+@pytest.mark.parametrize("qt", [NF4, FP4])
+def test_tiny_roundtrip_fp32(q, qt):
     wl = synth.WORKLOADS["tiny_roundtrip"]
     W = synth.weight(1024, 1024, wl.seed(synth.TID_W), "fp32")
-    _check_full(q, W, True)
-    _check_full(q, W, False)
+    _check_full(q, W, True, qt)
+    _check_full(q, W, False, qt)
 
 
-def test_attn_proj_bf16(q):
+@pytest.mark.parametrize("qt", [NF4, FP4])
+def test_attn_proj_bf16(q, qt):
     wl = synth.WORKLOADS["attn_proj_4096"]
     W = synth.weight(4096, 4096, wl.seed(synth.TID_W), "bf16")
-    _check_full(q, W, True)
+    _check_full(q, W, True, qt)
 
 
 @pytest.mark.parametrize("rows,cols", [(1, 64), (3, 6400), (7, 192), (5, 64 * 257)])
@@ -72,6 +82,57 @@ def test_ragged_shapes(q, rows, cols):
     """Single block, partial last DQ group (300 and 1285 scales), odd rows."""
     W = synth.weight(rows, cols, 77 + rows, "bf16")
     _check_full(q, W, True)
+    _check_full(q, W, True, FP4)
+
+
+def test_standalone_double_quantize(q):
+    """nf4_double_quantize on an absmax array (its own histogram pass) equals
+    the oracle, and the fused quantise + histogram path."""
+    W = synth.weight(300, 4096, 991, "bf16")
+    wq = q.quantize(W.cuda(), double_quant=True)
+    qa = torch.empty_like(wq.qabsmax)
+    sc = torch.empty_like(wq.dq_scale)
+    mu = torch.empty(4, dtype=torch.float32, device="cuda")[:1]
+    q.nf4_double_quantize(wq.absmax, qa, sc, mu)
+    assert q.qlora_check_status() == 0
+    a = oracle.block_absmax(W.float().numpy())
+    qa_r, s_r, mu_r = oracle.double_quantize(a)
+    assert np.array_equal(_np(qa), qa_r) and np.array_equal(_np(qa), _np(wq.qabsmax))
+    assert np.array_equal(_np(sc).view(np.uint32), s_r.view(np.uint32))
+    assert _np(mu)[0].view(np.uint32) == np.float32(mu_r).view(np.uint32)
+
+
+@pytest.mark.parametrize("splits", [(2, 4), (1, 3, 8)])
+def test_row_sharded_quantise_matches_whole(q, splits):
+    """A weight quantised in row shards -- each shard its own histogram, the
+    histograms summed, each shard's DQ finalised from the sum over the whole
+    count -- equals the whole weight's quantisation bit for bit (the shard
+    boundaries fall on groups of 256 scales: 4 rows of 4096 columns)."""
+    rows, cols = 8 * 4 + 3, 4096
+    W = synth.weight(rows, cols, 515, "bf16").cuda()
+    bounds = [0] + [4 * k for k in splits] + [rows]
+    whole = q.quantize(W, double_quant=True)
+    parts = []
+    hist = torch.zeros(256, dtype=torch.int64, device="cuda")
+    for r0, r1 in zip(bounds[:-1], bounds[1:]):
+        t = q.empty_quantized(r1 - r0, cols, W.device)
+        h = torch.empty(256, dtype=torch.int64, device="cuda")
+        q.qlora_quantize_4bit(W[r0:r1].contiguous(), t.packed, t.absmax, 0, h)
+        hist += h
+        parts.append(t)
+    n_total = rows * cols // 64
+    for t in parts:
+        q.nf4_double_quantize_hist(t.absmax, hist, n_total, t.qabsmax, t.dq_scale, t.dq_mean)
+    assert q.qlora_check_status() == 0
+    cat = lambda name: torch.cat([getattr(t, name) for t in parts])
+    assert torch.equal(cat("packed"), whole.packed)
+    assert torch.equal(cat("absmax"), whole.absmax)
+    assert torch.equal(cat("qabsmax"), whole.qabsmax)
+    assert torch.equal(cat("dq_scale"), whole.dq_scale)
+    for t in parts:
+        assert torch.equal(t.dq_mean, whole.dq_mean)
+    a = oracle.block_absmax(W.float().cpu().numpy())
+    assert np.float32(oracle.dq_mean(a)) == _np(whole.dq_mean)[0]
 
 
 def test_edge_values(q):
@@ -91,6 +152,7 @@ def test_edge_values(q):
         Wt = torch.from_numpy(W) if dt == "fp32" else torch.from_numpy(W).to(torch.bfloat16)
         _check_full(q, Wt, True)
         _check_full(q, Wt, False)
+        _check_full(q, Wt, False, FP4)
 
 
 def test_nonfinite_sets_status(q):
