@@ -234,6 +234,20 @@ int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_
 int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream);
 
 /*
+ * Merge the trained adapter into the base weight for export ([QE] "Why a
+ * 16-bit adapter will not fold into a 4-bit base": expand the base to 16
+ * bits first, then add; [LQ] "How LoRA Works": W' = W + (alpha/r) B A):
+ *   W_out[n, k] = RNbf16(RN32(w'[n, k] + RN32(s * sum_j B[n, j] A[j, k])))
+ *   w' = RNbf16(RN32(q[c] * a^)) (the nf4_dequantize values), s = alpha / r,
+ *   the sum over j accumulated in fp32 on tensor cores.
+ *   A device [r, K] bf16, B device [N, r] bf16, W_out device out [N, K] bf16.
+ * Constraints: r in {8,16,32,64,128}, alpha finite; one pass over the codes
+ * and one write of W_out.
+ */
+int qlora_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha,
+                void* W_out, qlora_stream_t stream);
+
+/*
  * QLoRA linear forward ([LQ] "How LoRA Works": W' = W + (alpha/r) B A;
  * [QE] "Why the expansion cannot be skipped": codes -> table -> scale ->
  * bf16 on chip -> tensor core):

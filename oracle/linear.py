@@ -67,3 +67,33 @@ def linear_bwd_adapters(X, dY, A, B, alpha: float, r: int):
     dA = s * ((dY @ B).T @ X)
     dB = s * (dY.T @ (X @ A.T))
     return dA, dB
+
+
+def round_bf16_f64(x) -> np.ndarray:
+    """fp64 -> bf16 round-to-nearest-even in one step (no fp32 in between);
+    returns the bf16 values as fp64.  bf16 keeps 8 significand bits: the top
+    1 + 7 of fp64's 53, so the low 45 bits of the fp64 pattern are dropped
+    with half rounding up and exact halves to an even kept part.  Finite
+    values of normal bf16 magnitude (>= 2^-126) or zero."""
+    u = np.asarray(x, dtype=np.float64).view(np.uint64)
+    keep = u >> np.uint64(45)
+    rest = u & np.uint64((1 << 45) - 1)
+    half = np.uint64(1 << 44)
+    up = (rest > half) | ((rest == half) & ((keep & np.uint64(1)) == np.uint64(1)))
+    return ((keep + up.astype(np.uint64)) << np.uint64(45)).view(np.float64)
+
+
+def merge(Wdeq, A, B, alpha: float, r: int) -> np.ndarray:
+    """The merged weight for export: RNbf16(W' + s B A), the sum in fp64 and
+    rounded once to bf16.
+
+    Page "QLoRA Explained", section "Why a 16-bit adapter will not fold into a
+    4-bit base": the adapter product is bf16 and cannot be added to 4-bit
+    codes, so the base is dequantised first (W' = the bf16 values of
+    dequantize) and the product added to it; page "LoRA vs QLoRA", section
+    "How LoRA Works": W + (alpha/r) B A with B d x r, A r x k.  Reading: the
+    result is stored in the compute type, bf16.
+    """
+    W, A, B = _f64(Wdeq), _f64(A), _f64(B)
+    s = float(alpha) / float(r)
+    return round_bf16_f64(W + s * (B @ A))

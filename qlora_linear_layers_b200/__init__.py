@@ -136,6 +136,15 @@ def nf4_dequantize(w: NF4Tensor, out: torch.Tensor, stream=None):
                "nf4_dequantize")
 
 
+def qlora_merge(w: NF4Tensor, A, B, alpha: float, out, stream=None):
+    """out[N, K] bf16 = RNbf16(deq(W) + (alpha / r) B A)."""
+    _need_cuda(A, B, out)
+    cw = w.c_struct()
+    _lib.check(_lib.load().qlora_merge(C.byref(cw), _ptr(A), _ptr(B), A.shape[0], float(alpha),
+                                       _ptr(out), _stream(stream)),
+               "qlora_merge")
+
+
 def qlora_linear_fwd(w: NF4Tensor, X, A, B, alpha: float, Y, T_save=None, ws=None, stream=None):
     _need_cuda(X, A, B, Y, T_save)
     M, r = X.shape[0], A.shape[0]
@@ -222,6 +231,12 @@ def quantize(W: torch.Tensor, double_quant: bool = True, quant_type: int = _lib.
 def dequantize(w: NF4Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=w.packed.device)
     nf4_dequantize(w, out, stream)
+    return out
+
+
+def merge(w: NF4Tensor, A, B, alpha: float, stream=None) -> torch.Tensor:
+    out = torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=w.packed.device)
+    qlora_merge(w, A, B, alpha, out, stream)
     return out
 
 

@@ -72,6 +72,7 @@ SIGNATURES = {
     "nf4_double_quantize": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nf4_double_quantize_hist": (_i32, [_vp, _i64, _vp, _i64, _i32, _vp, _vp, _vp, _vp]),
     "nf4_dequantize": (_i32, [C.POINTER(NF4Weight), _vp, _vp]),
+    "qlora_merge": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i32, _f32, _vp, _vp]),
     "qlora_linear_fwd": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
                                 _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i64, _vp, _vp, _i32, _f32,

@@ -326,6 +326,23 @@ int nf4_dequantize(const nf4_weight* w, void* W_out, qlora_stream_t stream) {
   return st;
 }
 
+int qlora_merge(const nf4_weight* w, const void* A, const void* B, int r, float alpha, void* W_out,
+                qlora_stream_t stream) {
+  int st = check_weight(w);
+  if (st) return st;
+  if (!A || !B || !W_out) return QLORA_ERR_INVALID_ARG;
+  if (!valid_rank(r) || !(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return QLORA_ERR_INVALID_ARG;
+  if (w->rows > (1 << 30) || w->cols > (1 << 30)) return QLORA_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+  DeviceInfo* d = nullptr;
+  st = current_device(&d);
+  if (st) return st;
+  launch_merge(w, A, B, r, alpha / (float)r, W_out, (cudaStream_t)stream);
+  st = launch_status();
+  if (!st) count_launches(1);
+  return st;
+}
+
 int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
                      int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {
@@ -379,8 +396,9 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);
-  // paired-SM tiles (256 weight rows) once there is more than one 128-row block
-  st = N > 128 ? launch_qlora_gemm_pair(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms)
+  // paired-SM tiles (256 weight rows, two token tiles each) once there is
+  // more than one 128-row block
+  st = N > 128 ? launch_qlora_gemm_dual(a, X, sT, RP, s, d->sms)
                : launch_qlora_gemm(MODE_NF4, a, X, sT, Bp, nullptr, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;

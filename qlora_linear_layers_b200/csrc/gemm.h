@@ -37,6 +37,12 @@ struct GemmArgs {
 int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
                            const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);
 
+// Forward NF4 GEMM on SM pairs with two token tiles per weight tile (the
+// weights of a stage are dequantised once into shared memory and feed two
+// 256-row x BM MMAs).  tok: [Mtok, Kc]; tokad: [Mtok, RP]; weights from `a`.
+int launch_qlora_gemm_dual(const GemmArgs& a, const void* tok, const void* tokad, int RP,
+                           cudaStream_t s, int num_sms);
+
 // tok: [Mtok, Kc]; tokad: [Mtok, RP]; wad: [Nout, RP]; w: [Nout, Kc] (MODE_BF16 only).
 int launch_qlora_gemm(int mode, const GemmArgs& a, const void* tok, const void* tokad,
                       const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);

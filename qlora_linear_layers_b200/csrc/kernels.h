@@ -29,6 +29,10 @@ int launch_double_quantize_from_hist(const float* absmax, int64_t n, const unsig
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms);
 
+// W_merged = RNbf16(deq(W) + s B A), [rows, cols] bf16 (merge.cu).
+void launch_merge(const nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
+                  cudaStream_t st);
+
 // All argument checks of qlora_linear_fwd except the workspace (capi.cu).
 int validate_fwd_args(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
                       int r, float alpha, const void* Y, const void* T_save);

@@ -606,3 +606,56 @@ def test_bf16_in_fp64_products_are_exact():
     got = float(np.dot(x, w))
     assert abs(Fraction(got) - exact) <= Fraction(1, 2 ** 40) * max(1, abs(exact))
     assert math.isfinite(got)
+
+
+# ---------------------------------------------------------------------------
+# Merge (base dequantised, then the adapter product added)
+# ---------------------------------------------------------------------------
+
+def test_round_bf16_f64_matches_torch_on_exact_fp32_values_and_ties():
+    """One-step fp64 -> bf16 rounding: equals torch's fp32 -> bf16 cast where
+    the fp64 value is an fp32 value, and breaks exact halves to even."""
+    rng = np.random.default_rng(41)
+    x = (rng.standard_normal(20000) * 0.05).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).float().numpy().astype(np.float64)
+    assert np.array_equal(oracle.round_bf16_f64(x.astype(np.float64)), want)
+    one = 1.0 + 2.0 ** -8                               # halfway between 1 and 1 + 2^-7
+    assert oracle.round_bf16_f64(np.array([one]))[0] == 1.0
+    assert oracle.round_bf16_f64(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+    assert oracle.round_bf16_f64(np.array([one + 2.0 ** -40]))[0] == 1.0 + 2.0 ** -7
+
+
+def test_merge_special_cases_and_orientation():
+    """B = 0 returns the dequantised weight; a rank-1 case worked by hand
+    fixes the orientation W[n, k] += s B[n] A[k]; the merged weight is within
+    half a bf16 ulp of the exact sum."""
+    rng = np.random.default_rng(42)
+    W = oracle.round_bf16((rng.standard_normal((6, 64)) * 0.02).astype(np.float32)).astype(np.float64)
+    A = rng.standard_normal((8, 64)) * 0.02
+    assert np.array_equal(oracle.merge(W, A, np.zeros((6, 8)), 16.0, 8), W)
+    A1 = np.zeros((1, 64)); A1[0, 5] = 0.5
+    B1 = np.zeros((6, 1)); B1[3, 0] = 0.25
+    M1 = oracle.merge(np.zeros((6, 64)), A1, B1, 4.0, 1)
+    assert M1[3, 5] == 4.0 * 0.25 * 0.5 and np.count_nonzero(M1) == 1
+    B = rng.standard_normal((6, 8)) * 0.02
+    Mg = oracle.merge(W, A, B, 16.0, 8)
+    exact = W + 2.0 * (B @ A)
+    ulp = np.spacing(np.abs(exact).astype(np.float32)).astype(np.float64) * 2.0 ** 16
+    assert np.all(np.abs(Mg - exact) <= ulp / 2)
+
+
+def test_merged_weight_reproduces_the_layer():
+    """X W_merged^T equals the layer's forward X W'^T + s (X A^T) B^T (pinned
+    against autograd above) up to the bf16 rounding of the merged weight."""
+    rng = np.random.default_rng(43)
+    N, K, M, r, alpha = 48, 128, 10, 16, 32.0
+    W = oracle.round_bf16((rng.standard_normal((N, K)) * 0.02).astype(np.float32)).astype(np.float64)
+    A = rng.standard_normal((r, K)) * 0.02
+    B = rng.standard_normal((N, r)) * 0.02
+    X = rng.standard_normal((M, K))
+    Y, _ = oracle.linear_fwd(X, W, A, B, alpha, r)
+    Ym = X @ oracle.merge(W, A, B, alpha, r).T
+    bound = np.abs(X) @ (np.abs(W + (alpha / r) * B @ A).T * 2.0 ** -8)
+    assert np.all(np.abs(Ym - Y) <= bound + 1e-15)
+    # and the adapter term is far above that bound (the check has teeth)
+    assert np.max(np.abs(X @ oracle.merge(W, A, B, alpha, r).T - (X @ W.T))) > 10 * np.max(bound)
