@@ -17,12 +17,11 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise.  Lanes own consecutive 16-byte chunks of the weight, so every
-// warp load instruction reads 512 contiguous bytes; a 64-weight block is 8
-// lanes (bf16) or 16 lanes (fp32), whose absmax is an integer max over |w|
-// bit patterns (exact; NaN/Inf show up as >= 0x7f800000) finished with
-// xor-shuffles inside the lane group.  Each lane issues the loads of four
-// chunks before computing any of them.
+// Quantise: one thread owns one 64-weight block (eight 16-byte bf16 loads or
+// sixteen fp32 ones, a 32-byte code store and its absmax), so the block max,
+// the reciprocal and the stores cost one thread's work per 64 weights, and a
+// warp's 32 blocks are contiguous.  absmax is an integer max over |w| bit
+// patterns (exact; NaN/Inf show up as >= 0x7f800000).
 //
 // Code of x = RN32(w / a):  x' = RN32(w * rcp(a)) with the hardware reciprocal
 // (at most 1 ulp off) is within 3.5 ulp of x.  A 64-entry bucket table over
@@ -30,24 +29,19 @@ namespace qnf4 {
 // a copy per lane, so the 32 lanes never meet on a bank) holds the single
 // threshold T that can fall in the bucket and the codes on either side of
 // it.  When x' is more than 8 ulp from T, x and x' are on the same side of
-// every threshold and the code follows from x' >= T; a lane with any x'
-// within 8 ulp of its T -- or whose block absmax is 0 or below 2^-125 --
-// redoes its own weights with the IEEE division (rare; out of line).
-// Thresholds sit >= 1e-4 from bucket edges (checked on the host), so x' may
-// pick the neighbouring bucket near an edge without effect.
+// every threshold and the code follows from x' >= T; a block with any x'
+// within 8 ulp of its T -- or whose absmax is 0 or below 2^-125 -- is redone
+// with the IEEE division (rare; out of line).  Thresholds sit >= 1e-4 from
+// bucket edges (checked on the host), so x' may pick the neighbouring bucket
+// near an edge without effect.
 //
 // With a histogram pointer the kernel also adds every block absmax into the
 // exponent histogram of the double quantisation (below): the significand of
-// each absmax, summed per fp32 exponent, warp-aggregated into shared memory
-// and then into the global 256-bin histogram.
+// each absmax, summed per fp32 exponent over the warp (match + reduce), then
+// into shared memory and, once per CTA, into the global 256-bin histogram.
 // ===========================================================================
 
-struct Bucket { float thr; uint32_t codes; };    // codes: lo (NF4), or lo | hi << 8
-
-__device__ __forceinline__ uint32_t bucket_index(float x) {
-  // round(16 x + 16) lands in the low mantissa bits of 16 x + 16 + 2^23
-  return __float_as_uint(fmaf(x, 16.0f, 8388624.0f)) & 63u;
-}
+struct Bucket { float thr; uint32_t codes; };    // codes: lo (code = rank), or lo | hi << 8
 
 __device__ __forceinline__ float rcp_approx(float a) {
   float r;
@@ -55,68 +49,87 @@ __device__ __forceinline__ float rcp_approx(float a) {
   return r;
 }
 
-// A 16-byte chunk of the weight.
-template <typename T> struct ChunkT;
-template <> struct ChunkT<__nv_bfloat16> {
-  static constexpr int kE = 8;                   // weights per chunk (bf16 pairs, element 2j low)
-  static constexpr int kL = 8;                   // chunks (lanes) per 64-weight block
-  __device__ __forceinline__ static uint32_t elem(const uint4& v, int i) {
-    const uint32_t w = i < 2 ? v.x : i < 4 ? v.y : i < 6 ? v.z : v.w;
-    return (i & 1) ? (w & 0xFFFF0000u) : (w << 16);
-  }
-  __device__ __forceinline__ static uint32_t absmax_bits(const uint4& v) {
-    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-    return max(m << 16, m & 0xFFFF0000u);
-  }
-};
-template <> struct ChunkT<float> {
-  static constexpr int kE = 4;
-  static constexpr int kL = 16;
-  __device__ __forceinline__ static uint32_t elem(const uint4& v, int i) {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-  }
-  __device__ __forceinline__ static uint32_t absmax_bits(const uint4& v) {
-    return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
-  }
-};
+// Shared-memory address of x's bucket entry in this lane's copy of the table
+// (bucket b, lane l at byte (b * 32 + l) * 8 from the table): 16 x + 16 + 2^23
+// rounds to 2^23 + round(16 x + 16), whose bit pattern is 0x4B000000 + b; the
+// shift by 8 drops the exponent bits and leaves b * 256.
+__device__ __forceinline__ uint32_t bucket_addr(float x, uint32_t lane_base) {
+  return (__float_as_uint(fmaf(x, 16.0f, 8388624.0f)) << 8) + lane_base;
+}
 
-// Bit position of weight i's code in the lane's packed word: element 2j goes
-// to the high nibble of byte j.
-__device__ __forceinline__ int nib_shift(int i) { return 8 * (i >> 1) + ((i & 1) ? 0 : 4); }
+__device__ __forceinline__ Bucket lds_bucket(uint32_t addr) {
+  Bucket b;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(b.thr), "=r"(b.codes) : "r"(addr));
+  return b;
+}
 
 template <bool MONO>
-__device__ __forceinline__ uint32_t code_of(float x, const Bucket* bkl, uint32_t& nearm) {
-  const Bucket b = bkl[bucket_index(x) * 32];
+__device__ __forceinline__ uint32_t code_of(float x, uint32_t lane_base, uint32_t& nearm) {
+  const Bucket b = lds_bucket(bucket_addr(x, lane_base));
   // same sign near T, so the bit patterns differ by the ulp distance
-  nearm = min(nearm, (uint32_t)(__float_as_int(x) - __float_as_int(b.thr) + 8));
+  nearm = __viaddmin_u32((uint32_t)(__float_as_int(x) - __float_as_int(b.thr)), 8u, nearm);
   const bool up = x >= b.thr;
   if (MONO) return b.codes + (up ? 1u : 0u);
   return up ? (b.codes >> 8) : (b.codes & 0xFFu);
 }
 
-// Exact codes of one chunk (x = RN32(w / a), or 0 for a zero block): the
-// rare path, kept out of line so the hot loop keeps its registers.
-template <typename T, bool MONO>
-__device__ __noinline__ uint32_t exact_codes(uint4 v, float a, bool zero_block, const Bucket* bkl) {
-  uint32_t out = 0, unused = 0;
-#pragma unroll
-  for (int i = 0; i < ChunkT<T>::kE; ++i) {
-    const float w = __uint_as_float(ChunkT<T>::elem(v, i));
-    const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
-    out += code_of<MONO>(x, bkl, unused) << nib_shift(i);
+// Weight i (0..63) of a block as an fp32 bit pattern, from the block's words.
+template <typename T> struct BlockWords;
+template <> struct BlockWords<__nv_bfloat16> {
+  static constexpr int kWords = 32;               // bf16 pairs, element 2j in the low half
+  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) {
+    return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
   }
-  return out;
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+    return max(m << 16, m & 0xFFFF0000u);
+  }
+};
+template <> struct BlockWords<float> {
+  static constexpr int kWords = 64;
+  __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) { return w[i]; }
+  __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kWords; ++j) m = max(m, w[j] & 0x7FFFFFFFu);
+    return m;
+  }
+};
+
+// Exact codes of block `blk` (x = RN32(w / a), or 0 for a zero block),
+// written straight to `packed`: the rare path, kept out of line so the hot
+// loop keeps its registers.
+template <typename T, bool MONO>
+__device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float a, bool zero_block,
+                                               uint32_t lane_base, uint8_t* packed) {
+  uint32_t out[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = 0u;
+  uint32_t unused = 0;
+  for (int i = 0; i < 64; ++i) {
+    float w;
+    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[blk * 64 + i]);
+    else w = reinterpret_cast<const float*>(W)[blk * 64 + i];
+    const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
+    const uint32_t code = code_of<MONO>(x, lane_base, unused);
+    const int sh = 8 * ((i >> 1) & 3) + ((i & 1) ? 0 : 4);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k == (i >> 3)) out[k] |= code << sh;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
 template <typename T, bool MONO, bool HIST>
 __global__ void __launch_bounds__(256)
-k_quantize(const uint4* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ packed,
+k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
            float* __restrict__ absmax, unsigned long long* __restrict__ hist, CodeTables tb,
            int* status) {
-  using C = ChunkT<T>;
-  constexpr int kU = 4;                          // chunks in flight per lane
-  __shared__ Bucket s_bk[64 * 32];               // bucket b, lane l at b * 32 + l
+  __shared__ __align__(8) Bucket s_bk[64 * 32];  // bucket b, lane l at b * 32 + l
   __shared__ unsigned long long s_hist[HIST ? 256 : 1];
   for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
     s_bk[i].thr = tb.bucket_thr[i >> 5];
@@ -127,48 +140,57 @@ k_quantize(const uint4* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ p
     for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0ull;
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const Bucket* bkl = s_bk + lane;
+  const uint32_t lane_base = smem_u32(s_bk) + (uint32_t)lane * 8u;
+  constexpr int kWords = BlockWords<T>::kWords;
   bool bad = false;
-  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t base = warp0 * (32 * kU); base < nchunks; base += nwarps * (32 * kU)) {
-    uint4 v[kU];
+  // warp-uniform loop (the histogram's match/reduce need whole warps)
+  const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  for (int64_t base = first; base < nblk; base += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t blk = base + lane;
+    const bool valid = blk < nblk;
+    uint32_t w[kWords];
+    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * (valid ? blk : 0);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t c = base + u * 32 + lane;
-      v[u] = c < nchunks ? __ldcs(W + c) : make_uint4(0u, 0u, 0u, 0u);
+    for (int k = 0; k < kWords / 4; ++k) {
+      const uint4 v = valid ? __ldcs(src + k) : make_uint4(0u, 0u, 0u, 0u);
+      w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
     }
+    uint32_t m = BlockWords<T>::absmax_bits(w);
+    if (m >= 0x7F800000u) { bad = true; m = 0; }
+    const float a = __uint_as_float(m);
+    if (valid) {
+      const bool exact_block = m < 0x01000000u;   // a == 0 or a < 2^-125
+      const float inv = exact_block ? 0.0f : rcp_approx(a);
+      uint32_t out[8];
+      uint32_t nearm = 0xFFFFFFFFu;               // min over the block of (ulp distance to T) + 8
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t c = base + u * 32 + lane;   // a lane group's chunks are all in or all out
-      uint32_t m = C::absmax_bits(v[u]);
+      for (int k = 0; k < 8; ++k) {
+        uint32_t o = 0;
 #pragma unroll
-      for (int o = 1; o < C::kL; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (m >= 0x7F800000u) { bad = true; m = 0; }
-      const float a = __uint_as_float(m);
-      const bool exact_all = m < 0x01000000u;   // a == 0 or a < 2^-125
-      const float inv = exact_all ? 0.0f : rcp_approx(a);
-      uint32_t nearm = 0xFFFFFFFFu, out = 0;
-#pragma unroll
-      for (int i = 0; i < C::kE; ++i) {
-        const float x = __fmul_rn(__uint_as_float(C::elem(v[u], i)), inv);
-        out += code_of<MONO>(x, bkl, nearm) << nib_shift(i);   // fields disjoint: add = or
+        for (int e = 0; e < 8; ++e) {
+          const int i = 8 * k + e;
+          const float x = __fmul_rn(__uint_as_float(BlockWords<T>::elem(w, i)), inv);
+          // element 2j -> high nibble of byte j (fields disjoint: add = or)
+          o += code_of<MONO>(x, lane_base, nearm) << (8 * (e >> 1) + ((e & 1) ? 0 : 4));
+        }
+        out[k] = o;
       }
-      if (exact_all || nearm <= 16u) out = exact_codes<T, MONO>(v[u], a, m == 0, bkl);
-      const bool lead = (lane & (C::kL - 1)) == 0;
-      if (c < nchunks) {
-        if (C::kE == 8) reinterpret_cast<uint32_t*>(packed)[c] = out;
-        else reinterpret_cast<uint16_t*>(packed)[c] = (uint16_t)out;
-        if (lead) absmax[c / C::kL] = a;
+      if (exact_block || nearm <= 16u) {
+        exact_block_codes<T, MONO>(W, blk, a, m == 0, lane_base, packed);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
+        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
       }
-      if (HIST) {
-        const bool add = lead && c < nchunks && m != 0u;
-        const uint32_t e = add ? (m >> 23) : 0xFFFFFFFFu;
-        const uint32_t mant = add ? ((m & 0x7FFFFFu) | (e ? 0x800000u : 0u)) : 0u;
-        const uint32_t grp = __match_any_sync(0xffffffffu, e);
-        const uint32_t sum = __reduce_add_sync(grp, mant);     // at most 4 terms below 2^24
-        if (add && lane == __ffs(grp) - 1) atomicAdd(&s_hist[e], (unsigned long long)sum);
-      }
+      absmax[blk] = a;
+    }
+    if (HIST) {
+      const bool add = valid && m != 0u;
+      const uint32_t e = add ? (m >> 23) : 0xFFFFFFFFu;
+      const uint32_t mant = add ? ((m & 0x7FFFFFu) | (e ? 0x800000u : 0u)) : 0u;
+      const uint32_t grp = __match_any_sync(0xffffffffu, e);
+      const uint32_t sum = __reduce_add_sync(grp, mant);       // < 32 * 2^24
+      if (add && lane == __ffs(grp) - 1) atomicAdd(&s_hist[e], (unsigned long long)sum);
     }
   }
   if (HIST) {
@@ -180,37 +202,36 @@ k_quantize(const uint4* __restrict__ W, int64_t nchunks, uint8_t* __restrict__ p
 }
 
 template <typename T, bool MONO>
-static void launch_quantize_t(const void* W, int64_t nchunks, uint8_t* packed, float* absmax,
+static void launch_quantize_t(const void* W, int64_t nblk, uint8_t* packed, float* absmax,
                               unsigned long long* hist, const CodeTables& tb, int* status,
-                              cudaStream_t s, int num_sms) {
-  constexpr int kThreads = 256, kPerCta = (kThreads / 32) * 32 * 4;   // chunks per CTA pass
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nchunks + kPerCta - 1) / kPerCta,
-                                                                 (int64_t)num_sms * 4));
+                              cudaStream_t s) {
+  constexpr int kThreads = 256;
+  // one block per thread: other CTAs' loads cover each block's compute
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nblk + kThreads - 1) / kThreads,
+                                                                 (int64_t)1 << 30));
   if (hist)
-    k_quantize<T, MONO, true><<<blocks, kThreads, 0, s>>>((const uint4*)W, nchunks, packed, absmax,
-                                                          hist, tb, status);
+    k_quantize<T, MONO, true><<<blocks, kThreads, 0, s>>>(W, nblk, packed, absmax, hist, tb, status);
   else
-    k_quantize<T, MONO, false><<<blocks, kThreads, 0, s>>>((const uint4*)W, nchunks, packed, absmax,
-                                                           nullptr, tb, status);
+    k_quantize<T, MONO, false><<<blocks, kThreads, 0, s>>>(W, nblk, packed, absmax, nullptr, tb, status);
 }
 
 int launch_quantize(const void* W, int dtype, int64_t n, int quant_type, uint8_t* packed,
                     float* absmax, unsigned long long* hist, int* status, cudaStream_t s,
                     int num_sms) {
+  (void)num_sms;
   const CodeTables& tb = host_tables(quant_type);
   int launched = 1;
   if (hist) {
     cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
     ++launched;
   }
-  const bool bf16 = dtype == QLORA_BF16;
-  const int64_t nchunks = bf16 ? n / 8 : n / 4;
-  if (bf16) {
-    if (tb.monotone) launch_quantize_t<__nv_bfloat16, true>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
-    else launch_quantize_t<__nv_bfloat16, false>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+  const int64_t nblk = n / 64;
+  if (dtype == QLORA_BF16) {
+    if (tb.monotone) launch_quantize_t<__nv_bfloat16, true>(W, nblk, packed, absmax, hist, tb, status, s);
+    else launch_quantize_t<__nv_bfloat16, false>(W, nblk, packed, absmax, hist, tb, status, s);
   } else {
-    if (tb.monotone) launch_quantize_t<float, true>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
-    else launch_quantize_t<float, false>(W, nchunks, packed, absmax, hist, tb, status, s, num_sms);
+    if (tb.monotone) launch_quantize_t<float, true>(W, nblk, packed, absmax, hist, tb, status, s);
+    else launch_quantize_t<float, false>(W, nblk, packed, absmax, hist, tb, status, s);
   }
   return launched;
 }
