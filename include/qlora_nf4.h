@@ -135,6 +135,14 @@ int nf4_code_thresholds(float* thresholds15);
 int qlora_code_table(int quant_type, float* table16);
 int qlora_code_thresholds(int quant_type, float* thresholds15, int* count);
 
+/* The double-quantisation mean from a complete exponent histogram over
+ * n_total absmax values (QLORA_DQ_HIST_BYTES of int64, host memory): the
+ * same exact rounding as the device, RN32(RN64(exact sum) / n_total), on
+ * the host -- for a caller that gathers shard histograms on the host.
+ * Returns QLORA_OK or QLORA_ERR_INVALID_ARG (null, n_total < 1, a negative
+ * bin). */
+int qlora_dq_mean_from_hist(const int64_t* hist, int64_t n_total, float* mean);
+
 /* Bytes of caller workspace needed by an operation (0 if none).
  *   QLORA_OP_DOUBLE_QUANT: M, K, r ignored; N = number of absmax values.
  *   QLORA_OP_FWD / QLORA_OP_BWD: layer with M tokens, weight N x K, rank r. */

@@ -67,6 +67,7 @@ SIGNATURES = {
     "qlora_code_table": (_i32, [_i32, C.POINTER(C.c_float)]),
     "qlora_code_thresholds": (_i32, [_i32, C.POINTER(C.c_float), C.POINTER(C.c_int)]),
     "qlora_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
+    "qlora_dq_mean_from_hist": (_i32, [C.POINTER(C.c_int64), _i64, C.POINTER(C.c_float)]),
     "nf4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp]),
     "qlora_quantize_4bit": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
     "nf4_double_quantize": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),

@@ -3,6 +3,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <cuda_runtime.h>
@@ -224,6 +225,50 @@ int qlora_code_thresholds(int quant_type, float* thresholds15, int* count) {
   const CodeTables& tb = host_tables(quant_type);
   std::memcpy(thresholds15, tb.t, (size_t)tb.nt * sizeof(float));
   *count = tb.nt;
+  return QLORA_OK;
+}
+
+// Host restatement of the device's exact mean: S = sum_e hist[e] *
+// 2^(max(e,1)-1) in units of 2^-149 as a 384-bit integer, rounded to the
+// nearest double (ties to even), divided by n in double, rounded to float.
+int qlora_dq_mean_from_hist(const int64_t* hist, int64_t n_total, float* mean) {
+  if (!hist || !mean || n_total < 1) return QLORA_ERR_INVALID_ARG;
+  constexpr int L = 13;                                   // 416 bits, little-endian words
+  uint32_t acc[L] = {};
+  for (int e = 0; e < 255; ++e) {
+    if (hist[e] < 0) return QLORA_ERR_INVALID_ARG;
+    if (hist[e] == 0) continue;
+    const int sh = (e > 0 ? e : 1) - 1;
+    const int w0 = sh >> 5, b = sh & 31;
+    // hist[e] << b spans at most three words
+    const unsigned __int128 v = (unsigned __int128)(uint64_t)hist[e] << b;
+    uint64_t carry = 0;
+    for (int k = 0; k < L - w0; ++k) {
+      const uint64_t add = k < 4 ? (uint64_t)(uint32_t)(v >> (32 * k)) : 0;
+      const uint64_t t = (uint64_t)acc[w0 + k] + add + carry;
+      acc[w0 + k] = (uint32_t)t;
+      carry = t >> 32;
+      if (k >= 3 && carry == 0) break;
+    }
+  }
+  int top = -1;
+  for (int w = L - 1; w >= 0 && top < 0; --w)
+    if (acc[w]) top = 32 * w + 31 - __builtin_clz(acc[w]);
+  auto bit = [&](int i) -> uint64_t { return (i >= 0 && i < 32 * L) ? (acc[i >> 5] >> (i & 31)) & 1u : 0u; };
+  double S = 0.0;
+  if (top >= 0) {
+    const int lo = top > 52 ? top - 52 : 0;               // the 53-bit significand is bits [lo, top]
+    uint64_t mant = 0;
+    for (int i = top; i >= lo; --i) mant = (mant << 1) | bit(i);
+    if (lo > 0) {
+      const uint64_t rbit = bit(lo - 1);
+      bool sticky = false;
+      for (int i = 0; i < lo - 1 && !sticky; ++i) sticky = bit(i) != 0;
+      if (rbit && (sticky || (mant & 1))) ++mant;
+    }
+    S = std::ldexp((double)mant, lo - 149);               // exact: mant <= 2^53
+  }
+  *mean = (float)(S / (double)n_total);
   return QLORA_OK;
 }
 

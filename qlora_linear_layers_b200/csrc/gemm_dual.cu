@@ -69,6 +69,11 @@ struct Smem {
 
 constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (the tensor core's operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -189,7 +194,10 @@ k_qlora_gemm_dual(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     const int row = quad * 32 + lane;                           // row within the CTA's 128
     const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
     const int64_t kb_per_row = p.Kc / 64;
-    struct Src { uint4 c[8]; float a_raw, sg; int qa; bool valid, ad; };
+    // What a converter needs of one stage, fetched two of its stages ahead:
+    // the row's 32 code bytes and scale inputs (an adapter stage's 128 bytes
+    // of B are read when it is converted: one stage in nk + RP/64).
+    struct Src { uint4 c0, c1; float sg; int qa; int n; bool valid, ad; int ks; };
     auto fetch = [&](uint32_t ai, Src& d) -> bool {
       const uint32_t lt = ai / (uint32_t)nsteps;
       const int ks = (int)(ai - lt * (uint32_t)nsteps);
@@ -198,60 +206,59 @@ k_qlora_gemm_dual(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
       const int n = (tile % n_pairs_n) * (2 * BN) + (int)rank * BN + row;
       d.valid = n < p.Nout;
       d.ad = ks >= nk;
-      const int64_t nn = d.valid ? n : 0;
-      if (d.ad) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.wad + nn * p.RP + (ks - nk) * BK);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) d.c[i] = __ldcg(src + i);
-      } else {
-        const uint4* codes = reinterpret_cast<const uint4*>(p.packed + nn * (p.Kc / 2)) + 2 * ks;
-        d.c[0] = __ldcg(codes);
-        d.c[1] = __ldcg(codes + 1);
-        const int64_t b = nn * kb_per_row + ks;
-        if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); d.a_raw = 0.f; }
-        else { d.a_raw = __ldcg(p.absmax + b); d.qa = 0; d.sg = 0.f; }
+      d.ks = ks;
+      d.n = d.valid ? n : 0;
+      if (!d.ad) {
+        const uint4* codes = reinterpret_cast<const uint4*>(p.packed + (int64_t)d.n * (p.Kc / 2)) + 2 * ks;
+        d.c0 = __ldcg(codes);
+        d.c1 = __ldcg(codes + 1);
+        const int64_t b = (int64_t)d.n * kb_per_row + ks;
+        if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); }
+        else { d.sg = __ldcg(p.absmax + b); d.qa = 0; }
       }
       return true;
     };
-    uint8_t* const arow = &S.a[0][0] + row * 128;
-    const int swz = row & 7;
-    Src cur, nxt;
+    const uint32_t arow = smem_u32(&S.a[0][0]) + (uint32_t)row * 128u;
+    const uint32_t swz = (uint32_t)(row & 7);
+    Src s0, s1, s2;
     uint32_t ai = par;
-    bool have = fetch(ai, cur);
-    while (have) {
-      const bool more = fetch(ai + 2, nxt);       // prefetch this warp's next stage
+    bool have0 = fetch(ai, s0);
+    bool have1 = have0 && fetch(ai + 2, s1);
+    while (have0) {
+      const bool have2 = have1 && fetch(ai + 4, s2);   // this warp's stage after next
       uint32_t v[32];
-      if (!cur.valid) {
+      if (!s0.valid) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0u;
-      } else if (cur.ad) {
+      } else if (s0.ad) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.wad + (int64_t)s0.n * p.RP + (s0.ks - nk) * BK);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          v[4 * i] = cur.c[i].x; v[4 * i + 1] = cur.c[i].y;
-          v[4 * i + 2] = cur.c[i].z; v[4 * i + 3] = cur.c[i].w;
+          const uint4 c = __ldcg(src + i);
+          v[4 * i] = c.x; v[4 * i + 1] = c.y; v[4 * i + 2] = c.z; v[4 * i + 3] = c.w;
         }
       } else {
         // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
-        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 128], cur.sg), mu) : cur.a_raw;
+        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[s0.qa + 128], s0.sg), mu) : s0.sg;
         const Lut l = build_lut(a, p.q);
-        const uint32_t wds[8] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w,
-                                 cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};
+        const uint32_t wds[8] = {s0.c0.x, s0.c0.y, s0.c0.z, s0.c0.w, s0.c1.x, s0.c1.y, s0.c1.z, s0.c1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
       }
       const int sa = ai % NS;
       if (!mbar_wait_cluster(&S.a_empty[sa], ((ai / NS) & 1) ^ 1, abort, p.status)) break;
       // 16-byte chunk j (K elements 8j..8j+7) of the row at chunk position j ^ (row & 7)
-      uint8_t* dst = arow + sa * A_BYTES;
+      const uint32_t dst = arow + (uint32_t)sa * (uint32_t)A_BYTES;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(dst + ((j ^ swz) << 4)) =
-            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        sts128(dst + ((((uint32_t)j) ^ swz) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.a_full[sa]), 0));
-      cur = nxt;
-      have = more;
+      s0 = s1;
+      s1 = s2;
+      have0 = have1;
+      have1 = have2;
       ai += 2;
     }
   } else {
@@ -271,28 +278,31 @@ k_qlora_gemm_dual(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
       // lane pairs (o, o+1) swap halves so each lane stores two adjacent
       // outputs of one token row: even lanes token m, odd lanes token m+1
       const int ocol = n0 + row_in_tile - (odd ? 1 : 0);
-      const int nchunk = BM / 16;
+      // 32 columns per TMEM round trip (BM is a multiple of 16: a last
+      // half-round of 16)
 #pragma unroll 1
       for (int t = 0; t < 2; ++t) {
 #pragma unroll 1
-        for (int c16 = 0; c16 < nchunk; ++c16) {
-          uint32_t v[16];
-          tmem_ld16(tmem + tmem_lane + (uint32_t)(t * ACC1_COL + c16 * 16), v);
+        for (int c0 = 0; c0 < BM; c0 += 32) {
+          const bool two = c0 + 16 < BM;
+          uint32_t v[32];
+          tmem_ld16(tmem + tmem_lane + (uint32_t)(t * ACC1_COL + c0), v);
+          if (two) tmem_ld16(tmem + tmem_lane + (uint32_t)(t * ACC1_COL + c0 + 16), v + 16);
           tmem_wait_ld();
-          if (t == 1 && c16 == nchunk - 1) {
+          if (t == 1 && c0 + 32 >= BM) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0);
           }
-          uint32_t pk[8];
+          uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < 16; ++j)
             pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          const int mfirst = m0 + t * BM + c16 * 16 + (odd ? 1 : 0);
-          const int rows_left = (ocol < p.Nout) ? p.Mtok - mfirst : 0;
+          const int mfirst = m0 + t * BM + c0 + (odd ? 1 : 0);
+          const int rows_left = (ocol < p.Nout) ? min(p.Mtok - mfirst, (two ? 32 : 16) - (odd ? 1 : 0)) : 0;
           uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + (int64_t)mfirst * p.Nout + ocol);
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
+          for (int c = 0; c < 32; c += 2) {
             const uint32_t mine = pk[c / 2];
             const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
             const uint32_t o = odd ? prmt(other, mine, 0x7632) : prmt(mine, other, 0x5410);

@@ -127,3 +127,35 @@ def test_validation_before_any_device_call(lib):
         _lib.QLORA_ERR_SHAPE
     assert lib.nf4_double_quantize_hist(fake, 512, None, 512, 256, fake, fake, fake, None) == \
         _lib.QLORA_ERR_INVALID_ARG
+
+
+def test_host_mean_from_histogram_matches_oracle(lib):
+    """qlora_dq_mean_from_hist (host) equals oracle.dq_mean bit for bit on
+    ordinary, extreme and degenerate absmax sets."""
+    rng = np.random.default_rng(77)
+
+    def hist_of(a):
+        u = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.int64)
+        e = u >> 23
+        m = (u & 0x7FFFFF) | np.where(e > 0, 0x800000, 0)
+        h = np.zeros(256, dtype=np.int64)
+        np.add.at(h, e, m)
+        return h
+
+    cases = [
+        np.abs(rng.standard_normal(100000)).astype(np.float32) * np.float32(0.05),
+        np.array([1e-45, 3e-39, 1e-30, 1.0, 3e38], dtype=np.float32),      # subnormal to huge
+        np.array([0.0, 0.0, 0.0], dtype=np.float32),
+        np.array([0.25], dtype=np.float32),
+        (np.abs(rng.standard_normal(4097)) * 10.0 ** rng.integers(-30, 30, 4097)).astype(np.float32),
+    ]
+    for a in cases:
+        h = hist_of(a)
+        mean = C.c_float(0.0)
+        assert lib.qlora_dq_mean_from_hist(h.ctypes.data_as(C.POINTER(C.c_int64)), a.size,
+                                           C.byref(mean)) == 0
+        assert np.float32(mean.value).view(np.uint32) == np.float32(oracle.dq_mean(a)).view(np.uint32)
+    h = np.zeros(256, dtype=np.int64)
+    h[3] = -1
+    assert lib.qlora_dq_mean_from_hist(h.ctypes.data_as(C.POINTER(C.c_int64)), 1, C.byref(mean)) == \
+        _lib.QLORA_ERR_INVALID_ARG
