@@ -67,9 +67,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the per-workload kernel timings after the step")
-    ap.add_argument("--case", choices=["fwd", "bwd", "quantize", "dequantize", "dq", "decode"],
+    ap.add_argument("--case", choices=["fwd", "bwd", "quantize", "dequantize", "dq", "decode", "merge"],
                     help="profiling aid: run one operation on one projection and exit")
     ap.add_argument("--proj", type=int, default=0, help="--case: projection 0 gate, 1 up, 2 down")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="--case: workload whose weight shape and rank to use (mlp_7b, decode_70b, "
+                         "attn_proj_4096, bwd_4096)")
     ap.add_argument("--tokens", type=int, default=2048, help="--case: token count")
     ap.add_argument("--repeat", type=int, default=3, help="--case: timed calls after one warm-up call")
     return ap.parse_args()
@@ -114,6 +117,12 @@ def dq_standalone_bytes(n):  # from an absmax array: read it twice (histogram, c
 def dequant_bytes(n):        # read codes + int8 scales + group scales, write bf16
     na = n // 64
     return n // 2 + na + 4 * ((na + 255) // 256) + 2 * n
+
+
+def merge_bytes(N, K, r):     # codes + int8 scales + group scales + A + B read, bf16 written
+    n = N * K
+    na = n // 64
+    return n // 2 + na + 4 * ((na + 255) // 256) + 2 * r * (N + K) + 2 * n
 
 
 def decode_bytes(M, N, K, r):
@@ -532,6 +541,12 @@ def workload_timings(q, lib, dev, pk):
             "dequantize": {"us": t_dd * 1e3, "GB/s": gbs(dequant_bytes(n), t_dd),
                            "frac_hbm": gbs(dequant_bytes(n), t_dd) / hbm, "bytes": dequant_bytes(n)},
         }
+        if not outliers:
+            # the merge for export: codes + scales + A + B read, bf16 written
+            t_m = _time_op(lambda: q.qlora_merge(wq, A, B, alpha, Wd), 10, flush)
+            nb = merge_bytes(N, K, r)
+            rec["merge"] = {"us": t_m * 1e3, "GB/s": gbs(nb, t_m), "frac_hbm": gbs(nb, t_m) / hbm,
+                            "bytes": nb}
         del W, Wd
         for m in (wl.decode_M if not outliers else (16,)):
             X = synth.activations(m, K, wl.seed(synth.TID_X) + m).to(dev)
@@ -545,6 +560,21 @@ def workload_timings(q, lib, dev, pk):
         torch.cuda.empty_cache()
     out["decode_70b"] = {"workload": wl.name, **dec}
     del ws, A, B
+    torch.cuda.empty_cache()
+
+    # ---- the merge on the 7B-class gate projection (r = 64)
+    wl = synth.WORKLOADS["mlp_7b"]
+    (N, K), r, alpha = wl.weights[0], wl.r, wl.alpha
+    W = synth.weight(N, K, wl.seed(synth.TID_W), "bf16").to(dev)
+    A = synth.activations(r, K, wl.seed(synth.TID_A), sigma=0.02).to(dev)
+    B = synth.activations(N, r, wl.seed(synth.TID_B), sigma=0.02).to(dev)
+    wq = q.quantize(W)
+    Wd = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    t_m = _time_op(lambda: q.qlora_merge(wq, A, B, alpha, Wd), 10, flush)
+    nb = merge_bytes(N, K, r)
+    out["mlp_7b_gate_merge"] = {"us": t_m * 1e3, "GB/s": gbs(nb, t_m), "frac_hbm": gbs(nb, t_m) / hbm,
+                                "bytes": nb, "shape": [N, K, r]}
+    del W, A, B, wq, Wd
     torch.cuda.empty_cache()
 
     # ---- the 4096^2 attention projection forward and the 4096^2 backward
@@ -724,9 +754,9 @@ def run_case(args):
     build()
     import qlora_linear_layers_b200 as q
     from qlora_linear_layers_b200 import _lib, synth
-    wl = synth.WORKLOADS[WORKLOAD]
-    N, K = wl.weights[args.proj]
-    M = DECODE_M if args.case == "decode" else args.tokens
+    wl = synth.WORKLOADS[args.workload]
+    N, K = wl.weights[min(args.proj, len(wl.weights) - 1)]
+    M = min(args.tokens, DECODE_M) if args.case == "decode" else args.tokens
     r, alpha = wl.r, wl.alpha
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(1234 + args.proj)
@@ -751,6 +781,7 @@ def run_case(args):
         "dq": lambda: q.nf4_double_quantize_hist(wq.absmax, hist, wq.absmax.numel(), wq.qabsmax,
                                                  wq.dq_scale, wq.dq_mean),
         "dequantize": lambda: q.nf4_dequantize(wq, Wd),
+        "merge": lambda: q.qlora_merge(wq, A, B, alpha, Wd),
     }
     torch.cuda.synchronize()
     ops[args.case]()                                  # warm-up call

@@ -69,6 +69,19 @@ struct Smem {
 
 constexpr size_t smem_bytes() { return sizeof(Smem) + 1024; }
 
+// L2 policy for the weight codes: keep them (a launch re-reads each code once
+// per round of token tiles, while the token stream passes through L2).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ldg_hint(const uint4* ptr, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(ptr), "l"(pol));
+  return v;
+}
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
@@ -194,6 +207,7 @@ k_qlora_gemm_dual(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     const int row = quad * 32 + lane;                           // row within the CTA's 128
     const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
     const int64_t kb_per_row = p.Kc / 64;
+    const uint64_t pol = policy_evict_last();
     // What a converter needs of one stage, fetched two of its stages ahead:
     // the row's 32 code bytes and scale inputs (an adapter stage's 128 bytes
     // of B are read when it is converted: one stage in nk + RP/64).
@@ -210,8 +224,8 @@ k_qlora_gemm_dual(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
       d.n = d.valid ? n : 0;
       if (!d.ad) {
         const uint4* codes = reinterpret_cast<const uint4*>(p.packed + (int64_t)d.n * (p.Kc / 2)) + 2 * ks;
-        d.c0 = __ldcg(codes);
-        d.c1 = __ldcg(codes + 1);
+        d.c0 = ldg_hint(codes, pol);
+        d.c1 = ldg_hint(codes + 1, pol);
         const int64_t b = (int64_t)d.n * kb_per_row + ks;
         if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); }
         else { d.sg = __ldcg(p.absmax + b); d.qa = 0; }

@@ -80,8 +80,15 @@ constexpr int kARows = 16;                       // adapter rows per row group
 constexpr int kWBytes = 16384;                   // 64 rows x 256 B of codes, or 8 x 16 A rows x 128 B
 // per stage: weights, then X of the stage's 8 blocks (8 * NT rows x 128 B each)
 template <int NT> __host__ __device__ constexpr int stage_bytes() { return kWBytes + kBlk * 1024 * NT; }
-// ring depth (fits beside the table and the reduction buffer)
-template <int NT> __host__ __device__ constexpr int n_stages() { return NT == 1 ? 6 : 4; }
+// Shared-memory map (shared-window addresses): [start, 64 KB) the small state
+// and, for one token tile, one ring stage; [64 KB, 128 KB) the pair table;
+// [128 KB, ...) the other ring stages.  The table's fixed address lets one
+// prmt build a lookup address (see the consumers).
+constexpr uint32_t kTableAddr = 0x10000;
+constexpr uint32_t kRingAddr = 0x20000;
+template <int NT> __host__ __device__ constexpr int n_stages_low() { return NT == 1 ? 1 : 0; }
+template <int NT> __host__ __device__ constexpr int n_stages_high() { return NT == 1 ? 4 : 3; }
+template <int NT> __host__ __device__ constexpr int n_stages() { return n_stages_low<NT>() + n_stages_high<NT>(); }
 constexpr int kMaxParts = 148;                   // ranges of the unit list (at most)
 
 struct GemvArgs {
@@ -98,17 +105,21 @@ struct GemvArgs {
   int nrg;                    // NF4 row groups: ceil(N / 64)
   int64_t U;                  // units: (nat + nrg) * spr
   int P;                      // ranges (CTAs): min(148, U)
+  uint32_t smem_base;         // shared-window address of dynamic shared memory
   float q[16];
 };
 
 template <int NT>
-struct GemvSmem {
-  uint8_t stage[n_stages<NT>()][stage_bytes<NT>()];   // 1024-aligned (128B-swizzled boxes)
+struct GemvSmem {                                // at the start of dynamic shared memory
   float red[kBlk][kRows * 16];                   // per-block sums of a piece
   float inv127[256];
   uint64_t full[n_stages<NT>()], empty[n_stages<NT>()];
   int abort;
 };
+// byte offset (from the start of dynamic shared memory) of the low ring stage
+template <int NT> __host__ __device__ constexpr uint32_t low_stage_off() {
+  return (uint32_t)((sizeof(GemvSmem<NT>) + 1023) / 1024 * 1024);
+}
 
 // Range (CTA) that owns unit x when U units are cut into P <= U ranges
 // start(j) = floor(j U / P); every range is non-empty.
@@ -132,6 +143,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) break;
 }
 
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // 16 bf16 of row `row` of a 128-byte-swizzled 64-column bf16 tile: logical
 // columns [16c, 16c+16) (16-byte chunks 2c and 2c+1, stored at chunk ^ (row & 7)).
 __device__ __forceinline__ void lds_row16(const uint8_t* tile, int row, int c, uint32_t (&w)[8]) {
@@ -148,18 +165,29 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
              const __grid_constant__ CUtensorMap tm_a,       // A as [K/64][r][64] bf16, box 64 x 16 x 8, 128B swizzle
              const __grid_constant__ CUtensorMap tm_x,       // X as [K/64][M][64] bf16, box 64 x 8*NT x 8, 128B swizzle
              const GemvArgs p) {
-  // byte-pair -> bf16 pair table, entry e replicated for lane l at e * 32 + l
-  __shared__ __align__(16) uint32_t tbl[256 * 32];
-  extern __shared__ uint8_t gsm_raw[];
-  GemvSmem<NT>& S =
-      *smem_align1024<GemvSmem<NT>>(gsm_raw);
+  extern __shared__ __align__(1024) uint8_t gsm_raw[];
+  const uint32_t base = smem_u32(gsm_raw);
+  if (base != p.smem_base) {                     // the map needs the base the host sized it for
+    if (threadIdx.x == 0) set_status(p.status, QLORA_ERR_CUDA);
+    return;
+  }
+  GemvSmem<NT>& S = *reinterpret_cast<GemvSmem<NT>*>(gsm_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kStages = n_stages<NT>();
   constexpr uint32_t kTx = stage_bytes<NT>();
+  auto stage_ptr = [&](int s) -> uint8_t* {
+    return s < n_stages_low<NT>() ? gsm_raw + low_stage_off<NT>() + s * stage_bytes<NT>()
+                                  : gsm_raw + (kRingAddr - base) + (s - n_stages_low<NT>()) * stage_bytes<NT>();
+  };
 
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-    const int e = i >> 5;
-    tbl[i] = pack_bf16x2(p.q[e >> 4], p.q[e & 15]);   // element 2j (high nibble) low half
+  // byte-pair -> bf16 pair table: entry e (a code byte) for lane l at shared
+  // address kTableAddr + e * 256 + l * 4 (a copy per lane: no bank conflicts)
+  {
+    uint32_t* tbl = reinterpret_cast<uint32_t*>(gsm_raw + (kTableAddr - base));
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+      const int e = i >> 5, l = i & 31;
+      tbl[e * 64 + l] = pack_bf16x2(p.q[e >> 4], p.q[e & 15]);   // element 2j (high nibble) low half
+    }
   }
   for (int i = threadIdx.x; i < 256; i += blockDim.x) S.inv127[i] = __fdiv_rn((float)(i - 128), 127.0f);   // entry c + 128: any int8 c
   if (threadIdx.x == 0) {
@@ -190,7 +218,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
         const int s = (int)(k % kStages);
         if (!(ok = mbar_wait(&S.empty[s], ((k / kStages) & 1) ^ 1, abort, p.status))) break;
         const int b = st * kBlk;
-        uint8_t* dst = S.stage[s];
+        uint8_t* dst = stage_ptr(s);
         mbar_arrive_expect_tx(&S.full[s], kTx);
         if (rgp < p.nat) {
           tma_load_3d(dst, &tm_a, &S.full[s], 0, rgp * kARows, b);
@@ -215,8 +243,9 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
   const int w = warp;
   const int j = w & (kBlk - 1), h = w >> 3;      // block of the stage, row half
   const int g = lane >> 2, c = lane & 3;
-  const uint32_t lane4 = (uint32_t)lane * 4;
-  const uint8_t* tb = reinterpret_cast<const uint8_t*>(tbl);
+  // prmt source of a lookup address: byte 0 = lane * 4, byte 2 = 1
+  // (kTableAddr), bytes 1 and 3 zero; the code byte goes to byte 1
+  const uint32_t tsrc = kTableAddr | ((uint32_t)lane * 4);
   const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
   const int NE = p.N + p.r;
   // codes: box (j >> 2), logical bytes [(j & 3) * 32 + 8c, +8) of a 128-byte row
@@ -313,7 +342,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     if (++pst == p.spr) { pst = 0; ++prgp; }
     const int s = (int)(k % kStages);
     if (!(ok = mbar_wait(&S.full[s], (k / kStages) & 1, abort, p.status))) break;
-    const uint8_t* sb = S.stage[s];
+    const uint8_t* sb = stage_ptr(s);
     const bool nf4 = rgp >= p.nat;
     if (b < p.nb && (nf4 || h == 0)) {
       uint32_t xw[NT][8];
@@ -335,15 +364,14 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
           for (int t = 0; t < 2; ++t) {
             const uint32_t vg = (kk < 2) ? wg[t].x : wg[t].y;
             const uint32_t vh = (kk < 2) ? wh[t].x : wh[t].y;
-            // table offset of a byte: (byte << 7) | lane * 4
-            const uint32_t og0 = ((kk & 1) ? (vg >> 9) : (vg << 7)) & 0x7F80u;
-            const uint32_t og1 = ((kk & 1) ? (vg >> 17) : (vg >> 1)) & 0x7F80u;
-            const uint32_t oh0 = ((kk & 1) ? (vh >> 9) : (vh << 7)) & 0x7F80u;
-            const uint32_t oh1 = ((kk & 1) ? (vh >> 17) : (vh >> 1)) & 0x7F80u;
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(tb + (og0 | lane4));
-            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(tb + (og1 | lane4));
-            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(tb + (oh0 | lane4));
-            const uint32_t a3 = *reinterpret_cast<const uint32_t*>(tb + (oh1 | lane4));
+            // lookup address kTableAddr + byte * 256 + lane * 4: one prmt
+            // (selector 0x76j4: tsrc byte 0, code byte j, tsrc bytes 2 and 3)
+            const uint32_t s0 = (kk & 1) ? 0x7624u : 0x7604u;   // byte 2kk of the lane's 8
+            const uint32_t s1 = (kk & 1) ? 0x7634u : 0x7614u;   // byte 2kk + 1
+            const uint32_t a0 = lds_u32(prmt(vg, tsrc, s0));
+            const uint32_t a2 = lds_u32(prmt(vg, tsrc, s1));
+            const uint32_t a1 = lds_u32(prmt(vh, tsrc, s0));
+            const uint32_t a3 = lds_u32(prmt(vh, tsrc, s1));
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               if (kk == 0) mma16816_z(cb[t][nt], a0, a1, a2, a3, xw[nt][0], xw[nt][1]);
@@ -506,11 +534,21 @@ Plan plan(int N, int K, int r) {
   return pl;
 }
 
+// Dynamic shared memory for the map above when it starts at shared address
+// `base` (the block's reserved shared memory; the kernel has no static
+// shared memory).
+template <int NT>
+constexpr int gemv_smem_bytes(uint32_t base) {
+  return (int)(kRingAddr - base) + n_stages_high<NT>() * stage_bytes<NT>();
+}
+static_assert(low_stage_off<1>() + stage_bytes<1>() + 1024 <= kTableAddr, "low stage below the table");
+static_assert(sizeof(GemvSmem<2>) + 1024 <= kTableAddr, "state below the table");
+static_assert(gemv_smem_bytes<1>(0) <= 232448 && gemv_smem_bytes<2>(0) <= 232448, "shared memory per CTA");
+
 template <bool DQ, int NT>
 void launch_gemv_kernel(const CUtensorMap& tw, const CUtensorMap& ta, const CUtensorMap& tx,
                         const GemvArgs& a, cudaStream_t st) {
-  constexpr int smem = (int)sizeof(GemvSmem<NT>) + 1024;
-  static_assert(smem + 256 * 32 * 4 <= 232448, "shared memory per CTA");
+  const int smem = gemv_smem_bytes<NT>(a.smem_base);
   static std::atomic<unsigned long long> attr_devs{0};
   set_smem_attr_once(k_qlora_gemv<DQ, NT>, smem, attr_devs);
   k_qlora_gemv<DQ, NT><<<a.P, kThreads, smem, st>>>(tw, ta, tx, a);
@@ -534,6 +572,16 @@ int launch_qlora_gemv(const nf4_weight* w, const void* X, int M, const void* A, 
   a.M = M; a.N = (int)w->rows; a.K = (int)w->cols; a.r = r;
   const Plan pl = plan(a.N, a.K, r);
   a.nb = pl.nb; a.spr = pl.spr; a.nat = pl.nat; a.nrg = pl.nrg; a.U = pl.U; a.P = pl.P;
+  {
+    // dynamic shared memory starts after the block's reserved shared memory
+    int dev = 0, reserved = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return -1;
+    }
+    a.smem_base = (uint32_t)reserved;
+  }
   for (int i = 0; i < 16; ++i) a.q[i] = q[i];
   const int NT = M <= 8 ? 1 : 2;
   CUtensorMap tw, ta, tx;
