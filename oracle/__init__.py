@@ -50,4 +50,5 @@ from .nf4 import (  # noqa: F401
     round_bf16,
     stored_bits_per_param,
 )
+from . import dropout  # noqa: F401
 from .linear import linear_fwd, linear_bwd, linear_bwd_adapters, merge, round_bf16_f64  # noqa: F401

@@ -659,3 +659,73 @@ def test_merged_weight_reproduces_the_layer():
     assert np.all(np.abs(Ym - Y) <= bound + 1e-15)
     # and the adapter term is far above that bound (the check has teeth)
     assert np.max(np.abs(X @ oracle.merge(W, A, B, alpha, r).T - (X @ W.T))) > 10 * np.max(bound)
+
+
+# ---------------------------------------------------------------------------
+# LoRA dropout (counter-based mask)
+# ---------------------------------------------------------------------------
+
+def test_philox4x64_matches_numpy():
+    """oracle.dropout.philox4x64_10 equals NumPy's Philox bit generator (the
+    same published generator; NumPy increments its counter before each block,
+    so its state c - 1 yields block c)."""
+    from oracle import dropout as D
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        key = [int(v) for v in rng.integers(0, 2 ** 63, 2)]
+        ctr = [int(v) for v in rng.integers(1, 2 ** 63, 4)]
+        bg = np.random.Philox(key=key, counter=[ctr[0] - 1, ctr[1], ctr[2], ctr[3]])
+        want = [int(v) for v in bg.random_raw(4)]
+        assert list(D.philox4x64_10(ctr, key)) == want
+    bg = np.random.Philox(key=[0, 0])
+    st = bg.state                                        # the counter's carry into word 1
+    st["state"]["counter"] = np.array([2 ** 64 - 1, 0, 0, 0], dtype=np.uint64)
+    st["buffer_pos"] = 4
+    bg.state = st
+    assert list(D.philox4x64_10((0, 1, 0, 0), (0, 0))) == [int(v) for v in bg.random_raw(4)]
+
+
+def test_dropout_mask_rate_and_p_zero():
+    from oracle import dropout as D
+    m = D.keep_mask(64, 256, 0.05, seed=12345)
+    n = m.size
+    assert abs(m.mean() - 0.95) < 4 * np.sqrt(0.05 * 0.95 / n)
+    assert not np.array_equal(m, D.keep_mask(64, 256, 0.05, seed=12346))
+    assert D.keep_mask(8, 64, 0.0, seed=1).all()
+    # p = 0: the layer is the plain layer
+    rng = np.random.default_rng(6)
+    X = oracle.round_bf16(rng.standard_normal((8, 64)).astype(np.float32))
+    W = rng.standard_normal((16, 64)) * 0.02
+    A = rng.standard_normal((8, 64)) * 0.02
+    B = rng.standard_normal((16, 8)) * 0.02
+    Y0, T0 = oracle.linear_fwd(X, W, A, B, 16.0, 8)
+    Y1, T1 = D.linear_fwd_dropout(X, W, A, B, 16.0, 8, np.ones((8, 64), bool), 0.0)
+    assert np.array_equal(Y0, Y1) and np.array_equal(T0, T1)
+
+
+def test_dropout_layer_vs_autograd():
+    """With p = 1/2 the kept inputs scale by exactly 2 (no rounding), so the
+    fp64 autograd of Y = X W^T + s ((D * 2 X) A^T) B^T pins the forward and
+    all three gradients of the dropout layer."""
+    from oracle import dropout as D
+    rng = np.random.default_rng(7)
+    M, K, N, r, alpha, p = 12, 64, 24, 8, 16.0, 0.5
+    X = oracle.round_bf16(rng.standard_normal((M, K)).astype(np.float32)).astype(np.float64)
+    W = rng.standard_normal((N, K)) * 0.02
+    A = rng.standard_normal((r, K)) * 0.02
+    B = rng.standard_normal((N, r)) * 0.02
+    dY = rng.standard_normal((M, N))
+    mask = D.keep_mask(M, K, p, seed=99)
+    assert D.keep_scale(p) == 2.0 and 0 < mask.mean() < 1
+    Xt = torch.tensor(X, requires_grad=True)
+    At = torch.tensor(A, requires_grad=True)
+    Bt = torch.tensor(B, requires_grad=True)
+    Dm = torch.tensor(mask.astype(np.float64))
+    Y = Xt @ torch.tensor(W).T + (alpha / r) * (((Dm * 2.0 * Xt) @ At.T) @ Bt.T)
+    Y.backward(torch.tensor(dY))
+    Yo, _ = D.linear_fwd_dropout(X, W, A, B, alpha, r, mask, p)
+    dX, dA, dB = D.linear_bwd_dropout(X, dY, W, A, B, alpha, r, mask, p)
+    np.testing.assert_allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dX, Xt.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dA, At.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dB, Bt.grad.numpy(), rtol=1e-12, atol=1e-13)
