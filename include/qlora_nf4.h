@@ -78,8 +78,24 @@ typedef enum { QLORA_QUANT_NF4 = 0, QLORA_QUANT_FP4 = 1 } qlora_quant_type;
 typedef enum {
   QLORA_OP_DOUBLE_QUANT = 0,
   QLORA_OP_FWD = 1,
-  QLORA_OP_BWD = 2
+  QLORA_OP_BWD = 2,
+  QLORA_OP_FWD_DROPOUT = 3,
+  QLORA_OP_BWD_DROPOUT = 4
 } qlora_op;
+
+/* LoRA dropout on the adapter's input ([QE] config walk-through:
+ * lora_dropout=0.05).  Element e = m * K + k of X is kept with probability
+ * 1 - p: Philox4x64-10 (Salmon et al., "Parallel Random Numbers: As Easy as
+ * 1, 2, 3", SC 2011) with key (seed, 0) and counter (e / 8, 0, 0, 0); word
+ * (e % 8) / 2 of the block, bits 40..63 (e even) or 16..39 (e odd), as a
+ * 24-bit uniform u; kept when u >= floor(p * 2^24 + 1/2).  Kept inputs are
+ * RNbf16(RN32(x * c)) with c = RN32(1 / RN32(1 - p)); the same mask is
+ * regenerated in the backward.  p in [0, 1); p = 0 is the plain layer. */
+typedef struct {
+  float p;
+  uint32_t reserved;      /* 0 */
+  uint64_t seed;
+} qlora_dropout;
 
 /*
  * A quantised frozen weight W[rows, cols] (rows = N output features,
@@ -290,6 +306,29 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY,
                      int64_t M, const void* A, const void* B, int r,
                      float alpha, const void* T, void* dX, void* dA, void* dB,
                      void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * The layer with LoRA dropout on the adapter's input (see qlora_dropout):
+ *   Y  = X deq(W)^T + s (X' A^T) B^T,   X' = dropout(X)
+ *   T_save = RNbf16(X' A^T)
+ *   dX = dY deq(W) + D * c * (s U A),  dA = s U^T X',  dB = s dY^T T
+ * with D the keep mask and c its scale.  Same arguments and constraints as
+ * qlora_linear_fwd / qlora_linear_bwd plus `dropout` (not null; p outside
+ * [0, 1) is QLORA_ERR_INVALID_ARG); workspaces from
+ * qlora_workspace_bytes(QLORA_OP_FWD_DROPOUT / QLORA_OP_BWD_DROPOUT, ...).
+ * Every token count runs the tensor-core GEMM (the decode kernel reads X once
+ * for base and adapter alike).  The backward's dX is the GEMM of dY deq(W)
+ * followed by a rank-r pass that adds the masked adapter term in place.
+ */
+int qlora_linear_fwd_dropout(const nf4_weight* w, const void* X, int64_t M,
+                             const void* A, const void* B, int r, float alpha,
+                             const qlora_dropout* dropout, void* Y, void* T_save,
+                             void* ws, size_t ws_bytes, qlora_stream_t stream);
+int qlora_linear_bwd_dropout(const nf4_weight* w, const void* X, const void* dY,
+                             int64_t M, const void* A, const void* B, int r,
+                             float alpha, const qlora_dropout* dropout, const void* T,
+                             void* dX, void* dA, void* dB, void* ws, size_t ws_bytes,
+                             qlora_stream_t stream);
 
 /*
  * Forward without a workspace argument, for callers that cannot allocate

@@ -17,9 +17,10 @@ Readings (the page names only the rate):
 * The mask is drawn from a counter-based generator so that the forward and
   the backward regenerate the same mask: Philox4x64-10 (Salmon, Moraes, Dror
   and Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), key
-  (seed, 0), counter (e // 4, 0, 0, 0) for element e = m * K + k of X, output
-  word e % 4.  An element is kept when the top 24 bits of its word are at
-  least round(p * 2^24).
+  (seed, 0), counter (e // 8, 0, 0, 0) for element e = m * K + k of X.  One
+  block's four 64-bit words serve eight elements: element e uses word
+  (e % 8) // 2, bits 40..63 for even e and bits 16..39 for odd e, as a
+  24-bit uniform u; the element is kept when u >= floor(p * 2^24 + 1/2).
 * X' is rounded to bf16 like every adapter operand: X' = RNbf16(RN32(x * c))
   with c = RN32(1 / RN32(1 - p)); dropped elements are 0.
 * The dropout gradient's factor is the same c: dX's adapter term is
@@ -65,8 +66,9 @@ def philox4x64_10(counter, key) -> tuple[int, int, int, int]:
 
 
 def keep_threshold(p: float) -> int:
-    """round(p * 2^24): words whose top 24 bits are below it are dropped."""
-    return int(round(float(np.float32(p)) * (1 << 24)))
+    """floor(RN32(p) * 2^24 + 1/2) (exact in fp64): 24-bit uniforms below it
+    are dropped."""
+    return int(np.floor(float(np.float32(p)) * (1 << 24) + 0.5))
 
 
 def keep_mask(M: int, K: int, p: float, seed: int) -> np.ndarray:
@@ -75,12 +77,13 @@ def keep_mask(M: int, K: int, p: float, seed: int) -> np.ndarray:
     thr = keep_threshold(p)
     n = M * K
     out = np.empty(n, dtype=bool)
-    for blk in range((n + 3) // 4):
+    for blk in range((n + 7) // 8):
         words = philox4x64_10((blk, 0, 0, 0), (seed, 0))
-        for i in range(4):
-            e = 4 * blk + i
+        for i in range(8):
+            e = 8 * blk + i
             if e < n:
-                out[e] = (words[i] >> 40) >= thr
+                u = (words[i // 2] >> (40 if i % 2 == 0 else 16)) & 0xFFFFFF
+                out[e] = u >= thr
     return out.reshape(M, K)
 
 

@@ -172,6 +172,37 @@ def qlora_linear_bwd(w: NF4Tensor, X, dY, A, B, alpha: float, dX, dA, dB, T=None
                "qlora_linear_bwd")
 
 
+def qlora_linear_fwd_dropout(w: NF4Tensor, X, A, B, alpha: float, p: float, seed: int, Y,
+                             T_save=None, ws=None, stream=None):
+    """The forward with LoRA dropout (rate p, Philox seed) on the adapter input."""
+    _need_cuda(X, A, B, Y, T_save)
+    M, r = X.shape[0], A.shape[0]
+    if ws is None:
+        ws = _workspace(workspace_bytes(_lib.QLORA_OP_FWD_DROPOUT, M, w.rows, w.cols, r), X.device)
+    cw = w.c_struct()
+    dr = _lib.Dropout(p=float(p), reserved=0, seed=int(seed))
+    _lib.check(_lib.load().qlora_linear_fwd_dropout(C.byref(cw), _ptr(X), M, _ptr(A), _ptr(B), r,
+                                                    float(alpha), C.byref(dr), _ptr(Y), _ptr(T_save),
+                                                    _ptr(ws), ws.numel(), _stream(stream)),
+               "qlora_linear_fwd_dropout")
+
+
+def qlora_linear_bwd_dropout(w: NF4Tensor, X, dY, A, B, alpha: float, p: float, seed: int, dX, dA,
+                             dB, T=None, ws=None, stream=None):
+    """The backward with LoRA dropout; the mask is regenerated from (p, seed)."""
+    _need_cuda(X, dY, A, B, dX, dA, dB, T)
+    M, r = X.shape[0], A.shape[0]
+    if ws is None:
+        ws = _workspace(workspace_bytes(_lib.QLORA_OP_BWD_DROPOUT, M, w.rows, w.cols, r), X.device)
+    cw = w.c_struct()
+    dr = _lib.Dropout(p=float(p), reserved=0, seed=int(seed))
+    _lib.check(_lib.load().qlora_linear_bwd_dropout(C.byref(cw), _ptr(X), _ptr(dY), M, _ptr(A),
+                                                    _ptr(B), r, float(alpha), C.byref(dr), _ptr(T),
+                                                    _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                                                    ws.numel(), _stream(stream)),
+               "qlora_linear_bwd_dropout")
+
+
 def qlora_check_status(stream=None) -> int:
     """Synchronise the stream; return and clear the device status word."""
     return int(_lib.load().qlora_check_status(_stream(stream)))
@@ -246,6 +277,24 @@ def linear_fwd(w: NF4Tensor, X, A, B, alpha: float, save_T: bool = True, stream=
     T = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_T else None
     qlora_linear_fwd(w, X, A, B, alpha, Y, T, stream=stream)
     return Y, T
+
+
+def linear_fwd_dropout(w: NF4Tensor, X, A, B, alpha: float, p: float, seed: int,
+                       save_T: bool = True, stream=None):
+    M, r = X.shape[0], A.shape[0]
+    Y = torch.empty(M, w.rows, dtype=torch.bfloat16, device=X.device)
+    T = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_T else None
+    qlora_linear_fwd_dropout(w, X, A, B, alpha, p, seed, Y, T, stream=stream)
+    return Y, T
+
+
+def linear_bwd_dropout(w: NF4Tensor, X, dY, A, B, alpha: float, p: float, seed: int, T=None,
+                       stream=None):
+    dX = torch.empty_like(X)
+    dA = torch.empty_like(A)
+    dB = torch.empty_like(B)
+    qlora_linear_bwd_dropout(w, X, dY, A, B, alpha, p, seed, dX, dA, dB, T=T, stream=stream)
+    return dX, dA, dB
 
 
 def linear_bwd(w: NF4Tensor, X, dY, A, B, alpha: float, T=None, stream=None):

@@ -33,6 +33,8 @@ QLORA_DQ_HIST_BYTES = 2048
 QLORA_OP_DOUBLE_QUANT = 0
 QLORA_OP_FWD = 1
 QLORA_OP_BWD = 2
+QLORA_OP_FWD_DROPOUT = 3
+QLORA_OP_BWD_DROPOUT = 4
 
 QLORA_FWD_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -57,6 +59,11 @@ class NF4Weight(C.Structure):
     ]
 
 
+class Dropout(C.Structure):
+    """Mirror of `qlora_dropout` in include/qlora_nf4.h."""
+    _fields_ = [("p", C.c_float), ("reserved", C.c_uint32), ("seed", C.c_uint64)]
+
+
 SIGNATURES = {
     "qlora_abi_version": (_i32, []),
     "qlora_kernel_launches": (C.c_uint64, []),
@@ -78,6 +85,10 @@ SIGNATURES = {
                                 _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_bwd": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i64, _vp, _vp, _i32, _f32,
                                 _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_fwd_dropout": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
+                                        C.POINTER(Dropout), _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd_dropout": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i64, _vp, _vp, _i32, _f32,
+                                        C.POINTER(Dropout), _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_fwd_noalloc": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
                                         _vp, _vp, _vp]),
     "qlora_check_status": (_i32, [_vp]),

@@ -70,11 +70,11 @@ int padded_rank(int r) { return r <= 64 ? 64 : 128; }
 struct FwdWs {
   size_t sT, Bpad, part, gemv, total;
 };
-FwdWs fwd_ws(int64_t M, int64_t N, int64_t K, int r) {
+FwdWs fwd_ws(int64_t M, int64_t N, int64_t K, int r, bool gemm_path = false) {
   FwdWs w{};
   const int RP = padded_rank(r);
   size_t off = 0;
-  if (M <= kDecodeMaxTokens) {   // decode path: only the GEMV's partial sums
+  if (M <= kDecodeMaxTokens && !gemm_path) {   // decode path: only the GEMV's partial sums
     w.gemv = 0;
     w.total = align256(gemv_workspace_bytes((int)M, (int)N, (int)K, r));
     return w;
@@ -281,8 +281,12 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
       if (K < 1) return 0;
       return fwd_ws(M, N, K, r).total;
     case QLORA_OP_BWD:
+    case QLORA_OP_BWD_DROPOUT:
       if (M < 1 || N < 1 || K < 1 || !valid_rank(r)) return 0;
       return bwd_ws(M, N, K, r).total;
+    case QLORA_OP_FWD_DROPOUT:
+      if (M < 1 || N < 1 || K < 1 || !valid_rank(r)) return 0;
+      return fwd_ws(M, N, K, r, true).total;
     default: return 0;
   }
 }
@@ -388,13 +392,16 @@ int qlora_merge(const nf4_weight* w, const void* A, const void* B, int r, float 
   return st;
 }
 
-int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
-                     int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
-                     qlora_stream_t stream) {
+static int fwd_impl(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
+                    int r, float alpha, const Dropout* drop, void* Y, void* T_save, void* ws,
+                    size_t ws_bytes, qlora_stream_t stream) {
   int st = validate_fwd_args(w, X, M, A, B, r, alpha, Y, T_save);
   if (st) return st;
   const int64_t N = w->rows, K = w->cols;
-  const FwdWs lay = fwd_ws(M, N, K, r);
+  // dropout applies to the adapter's input only: the decode kernel, which
+  // reads X once for both, is left to the plain layer
+  const bool gemm_path = drop != nullptr;
+  const FwdWs lay = fwd_ws(M, N, K, r, gemm_path);
   if (!ws || ws_bytes < lay.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   DeviceInfo* d = nullptr;
@@ -404,7 +411,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   const int RP = padded_rank(r);
   const float scale = alpha / (float)r;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  if (M <= kDecodeMaxTokens) {
+  if (M <= kDecodeMaxTokens && !gemm_path) {
     // decode-sized call: HBM-bound GEMV on the warp-level tensor cores
     const int n = launch_qlora_gemv(w, X, (int)M, A, B, r, scale, Y, T_save,
                                     reinterpret_cast<float*>(wsb + lay.gemv), host_tables(w->quant_type).q,
@@ -423,7 +430,7 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
     ++n;
   }
   n += launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, sT, T_save,
-                        reinterpret_cast<float*>(wsb + lay.part), s);
+                        reinterpret_cast<float*>(wsb + lay.part), s, drop);
   GemmArgs a{};
   a.packed = w->packed;
   a.absmax = w->absmax;
@@ -452,9 +459,9 @@ int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* 
   return st;
 }
 
-int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
-                     const void* B, int r, float alpha, const void* T, void* dX, void* dA,
-                     void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+static int bwd_impl(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
+                    const void* B, int r, float alpha, const Dropout* drop, const void* T, void* dX,
+                    void* dA, void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
   int st = check_weight(w);
   if (st) return st;
   if (!X || !dY || !A || !B || !dX || !dA || !dB) return QLORA_ERR_INVALID_ARG;
@@ -481,7 +488,7 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   int n = 7;   // dequant_t, transpose_pad, GEMM, 2 x (partials + reduce)
   if (!T) {
     n += launch_lora_down(X, A, (int)M, (int)K, r, RP, scale, nullptr, Tw,
-                          reinterpret_cast<float*>(wsb + lay.pT), s);
+                          reinterpret_cast<float*>(wsb + lay.pT), s, drop);
     T = Tw;
   }
   n += launch_lora_u(dY, B, (int)M, (int)N, r, RP, scale, sU, reinterpret_cast<float*>(wsb + lay.pU), s);
@@ -493,7 +500,10 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
   a.wad = static_cast<const __nv_bfloat16*>(At);
   a.RP = RP;
   a.Mtok = (int)M; a.Nout = (int)K; a.Kc = (int)N;
-  a.na = RP / 64;
+  // with dropout the adapter term needs the keep mask: the GEMM writes dY W'
+  // alone and a rank-r pass adds D * c * (s U A)
+  const bool dropping = drop && drop->on;
+  a.na = dropping ? 0 : RP / 64;
   a.status = d->status;
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
@@ -502,14 +512,61 @@ int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t
                : launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;
+  if (dropping) {
+    launch_rank_add(sU, RP, A, r, (int)M, (int)K, dX, *drop, s);
+    ++n;
+  }
   // dA[r, K] = (s U)^T X ;  dB[N, r] = s dY^T T
   launch_atb(sU, RP, r, X, (int)K, (int)K, (int)M, 1.0f, dA, reinterpret_cast<float*>(wsb + lay.pA),
-             d->sms, s);
+             d->sms, s, drop);
   launch_atb(dY, (int)N, (int)N, T, r, r, (int)M, scale, dB, reinterpret_cast<float*>(wsb + lay.pB),
              d->sms, s);
   st = launch_status();
   if (!st) count_launches(n);
   return st;
+}
+
+int qlora_linear_fwd(const nf4_weight* w, const void* X, int64_t M, const void* A, const void* B,
+                     int r, float alpha, void* Y, void* T_save, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
+  return fwd_impl(w, X, M, A, B, r, alpha, nullptr, Y, T_save, ws, ws_bytes, stream);
+}
+
+int qlora_linear_bwd(const nf4_weight* w, const void* X, const void* dY, int64_t M, const void* A,
+                     const void* B, int r, float alpha, const void* T, void* dX, void* dA,
+                     void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  return bwd_impl(w, X, dY, M, A, B, r, alpha, nullptr, T, dX, dA, dB, ws, ws_bytes, stream);
+}
+
+// Dropout parameters -> the kernels' form; QLORA_OK with *on = 0 for p == 0.
+static int make_dropout(const qlora_dropout* dp, Dropout* out) {
+  if (!dp) return QLORA_ERR_INVALID_ARG;
+  const float p = dp->p;
+  if (!(p >= 0.0f && p < 1.0f)) return QLORA_ERR_INVALID_ARG;
+  out->seed = dp->seed;
+  out->thr = (uint32_t)std::floor((double)p * 16777216.0 + 0.5);
+  out->scale = 1.0f / (1.0f - p);
+  out->on = out->thr != 0 ? 1 : 0;
+  return QLORA_OK;
+}
+
+int qlora_linear_fwd_dropout(const nf4_weight* w, const void* X, int64_t M, const void* A,
+                             const void* B, int r, float alpha, const qlora_dropout* dropout,
+                             void* Y, void* T_save, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  Dropout dr{};
+  const int st = make_dropout(dropout, &dr);
+  if (st) return st;
+  return fwd_impl(w, X, M, A, B, r, alpha, &dr, Y, T_save, ws, ws_bytes, stream);
+}
+
+int qlora_linear_bwd_dropout(const nf4_weight* w, const void* X, const void* dY, int64_t M,
+                             const void* A, const void* B, int r, float alpha,
+                             const qlora_dropout* dropout, const void* T, void* dX, void* dA,
+                             void* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  Dropout dr{};
+  const int st = make_dropout(dropout, &dr);
+  if (st) return st;
+  return bwd_impl(w, X, dY, M, A, B, r, alpha, &dr, T, dX, dA, dB, ws, ws_bytes, stream);
 }
 
 int qlora_check_status(qlora_stream_t stream) {

@@ -75,6 +75,49 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// LoRA dropout mask: Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+// Random Numbers: As Easy as 1, 2, 3", SC 2011) with key (seed, 0) and
+// counter (e / 8, 0, 0, 0) for element e = m * K + k of the adapter input;
+// element e uses word (e % 8) / 2 of the block, bits 40..63 (e even) or
+// 16..39 (e odd), as a 24-bit uniform, kept when >= thr.
+// ---------------------------------------------------------------------------
+struct Dropout {
+  uint64_t seed;
+  uint32_t thr;      // floor(p * 2^24 + 1/2); 0 keeps everything
+  float scale;       // RN32(1 / RN32(1 - p))
+  int on;
+};
+
+__device__ __forceinline__ void philox4x64_10(uint64_t& c0, uint64_t& c1, uint64_t& c2, uint64_t& c3,
+                                              uint64_t k0, uint64_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B97F4A7C15ull;
+      k1 += 0xBB67AE8584CAA73Bull;
+    }
+    const uint64_t hi0 = __umul64hi(0xD2E7470EE14C6C93ull, c0), lo0 = 0xD2E7470EE14C6C93ull * c0;
+    const uint64_t hi1 = __umul64hi(0xCA5A826395121157ull, c2), lo1 = 0xCA5A826395121157ull * c2;
+    const uint64_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+  }
+}
+
+// Keep bits of elements 8 blk .. 8 blk + 7 (bit i: element 8 blk + i).
+__device__ __forceinline__ uint32_t dropout_keep8(uint64_t blk, uint64_t seed, uint32_t thr) {
+  uint64_t w0 = blk, w1 = 0, w2 = 0, w3 = 0;
+  philox4x64_10(w0, w1, w2, w3, seed, 0);
+  const uint64_t w[4] = {w0, w1, w2, w3};
+  uint32_t bits = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t u = (uint32_t)(w[i >> 1] >> ((i & 1) ? 16 : 40)) & 0xFFFFFFu;
+    bits |= (u >= thr ? 1u : 0u) << i;
+  }
+  return bits;
+}
+
+// ---------------------------------------------------------------------------
 // Small bit helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -92,6 +135,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Dropout on 8 consecutive bf16 (element i in half i % 2 of word i / 2):
+// kept -> RNbf16(RN32(x * scale)), dropped -> 0.
+__device__ __forceinline__ uint4 dropout8(uint4 v, uint32_t bits, float scale) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t pk = pack_bf16x2(__fmul_rn(bf16_lo(w[j]), scale), __fmul_rn(bf16_hi(w[j]), scale));
+    const uint32_t keep = ((bits >> (2 * j)) & 1u ? 0x0000FFFFu : 0u) | ((bits >> (2 * j + 1)) & 1u ? 0xFFFF0000u : 0u);
+    w[j] = pk & keep;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 // The first 1024-byte-aligned address at or after a dynamic shared array,
 // reached by offsetting the array itself so the compiler keeps shared-space

@@ -75,8 +75,12 @@ bool make_tmap_3d(CUtensorMap* tm, const void* base, bool bf16, const uint64_t d
 //   T_save[M, r]  = RNbf16(T)      (if not null)
 // `part` holds skinny_workspace_bytes(M, K, RP) bytes of fp32 partial sums.
 // Returns the number of kernels launched.
+struct Dropout;
+// With `drop` (LoRA dropout on X, may be null), T = X' A^T with X' the
+// dropped-out input.
 int launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
-                     void* sT_pad, void* T_save, float* part, cudaStream_t st);
+                     void* sT_pad, void* T_save, float* part, cudaStream_t st,
+                     const Dropout* drop = nullptr);
 size_t skinny_workspace_bytes(int M, int L, int RP);
 
 // U = dY B:  sU_pad[M, RP] = RNbf16(s * U), zero beyond r.
@@ -85,8 +89,15 @@ int launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, fl
 
 // C[Rdim, Cdim] = RNbf16(s * P^T Q) over M token rows, split over the tokens
 // into fixed chunks summed in order; `part` holds atb_workspace_floats floats.
+// With `dropq`, Q (the adapter input X) is dropped out on load.
 void launch_atb(const void* P, int ldp, int Rdim, const void* Q, int ldq, int Cdim, int M, float s,
-                void* out, float* part, int num_sms, cudaStream_t st);
+                void* out, float* part, int num_sms, cudaStream_t st, const Dropout* dropq = nullptr);
+
+// Y[M, K] (bf16, in place) += D * c * (Bm[M, :r] A[r, K]) with D the dropout
+// keep mask of Y's elements (drop.on == 0: no mask, c = 1): the adapter term
+// of dX under LoRA dropout.
+void launch_rank_add(const void* Bm, int ldb, const void* A, int r, int M, int K, void* Y,
+                     const Dropout& drop, cudaStream_t st);
 size_t atb_workspace_floats(int Rdim, int Cdim, int M);
 
 // Wt[K, N] = deq(W)^T (bf16, the values of nf4_dequantize).

@@ -66,11 +66,11 @@ __device__ __forceinline__ uint32_t swzw(int row, int col) {
 // several: fp32 partials part[split][M][RP], summed in order by
 // k_skinny_reduce.
 // ===========================================================================
-template <int RP, bool BT>
+template <int RP, bool BT, bool DROP>
 __global__ void __launch_bounds__(256)
 k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restrict__ R, int M,
               int L, int r, float s, int chunks_per_split, __nv_bfloat16* __restrict__ Ss,
-              __nv_bfloat16* __restrict__ Sraw, float* __restrict__ part) {
+              __nv_bfloat16* __restrict__ Sraw, float* __restrict__ part, Dropout drop) {
   constexpr int TM = 128, KC = 64, STG = 3;
   constexpr int XB = TM * KC * 2, AB = RP * KC * 2;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -125,6 +125,20 @@ k_lora_skinny(const __nv_bfloat16* __restrict__ Z, const __nv_bfloat16* __restri
     cp_async_commit();
     const uint8_t* xs = sm + (kc % STG) * (XB + AB);
     const uint8_t* as = xs + XB;
+    if (DROP) {
+      // LoRA dropout on this stage's rows of Z (the adapter input X)
+      uint8_t* xw = sm + (kc % STG) * (XB + AB);
+      for (int ci = tid; ci < TM * 8; ci += 256) {
+        const int row = ci >> 3, ch = ci & 7;
+        const int m = m0 + row, l = (kc0 + kc) * KC + ch * 8;
+        if (m < M && l < L) {
+          uint4* q = reinterpret_cast<uint4*>(xw + swz64(row, ch * 8));
+          *q = dropout8(*q, dropout_keep8(((uint64_t)m * (uint64_t)L + (uint64_t)l) >> 3, drop.seed, drop.thr),
+                        drop.scale);
+        }
+      }
+      __syncthreads();
+    }
 #pragma unroll
     for (int k16 = 0; k16 < KC / 16; ++k16) {
       uint32_t a0, a1, a2, a3;
@@ -212,19 +226,27 @@ size_t skinny_workspace_bytes(int M, int L, int RP) {
   return sp > 1 ? (size_t)sp * M * RP * 4 : 0;
 }
 
-template <int RP, bool BT>
-static void launch_skinny(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
-                          void* Sraw, float* part, cudaStream_t st) {
+template <int RP, bool BT, bool DROP>
+static void launch_skinny_t(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
+                            void* Sraw, float* part, const Dropout& drop, cudaStream_t st) {
   constexpr int smem = 3 * (128 * 64 * 2 + RP * 64 * 2);
   static std::atomic<unsigned long long> attr_devs{0};
-  set_smem_attr_once(k_lora_skinny<RP, BT>, smem, attr_devs);
+  set_smem_attr_once(k_lora_skinny<RP, BT, DROP>, smem, attr_devs);
   const int splits = skinny_splits(M, L);
   const int nkc = (L + 63) / 64;
   const int cps = (nkc + splits - 1) / splits;
   const dim3 grid((M + 127) / 128, splits);
-  k_lora_skinny<RP, BT><<<grid, 256, smem, st>>>(
+  k_lora_skinny<RP, BT, DROP><<<grid, 256, smem, st>>>(
       (const __nv_bfloat16*)Z, (const __nv_bfloat16*)R, M, L, r, s, cps, (__nv_bfloat16*)Ss,
-      (__nv_bfloat16*)Sraw, part);
+      (__nv_bfloat16*)Sraw, part, drop);
+}
+
+template <int RP, bool BT>
+static void launch_skinny(const void* Z, const void* R, int M, int L, int r, float s, void* Ss,
+                          void* Sraw, float* part, const Dropout& drop, cudaStream_t st) {
+  if (drop.on) launch_skinny_t<RP, BT, true>(Z, R, M, L, r, s, Ss, Sraw, part, drop, st);
+  else launch_skinny_t<RP, BT, false>(Z, R, M, L, r, s, Ss, Sraw, part, drop, st);
+  const int splits = skinny_splits(M, L);
   if (splits > 1) {
     const int64_t total = (int64_t)M * RP / 2;
     const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 8);
@@ -235,16 +257,18 @@ static void launch_skinny(const void* Z, const void* R, int M, int L, int r, flo
 
 // Returns the number of kernels launched.
 int launch_lora_down(const void* X, const void* A, int M, int K, int r, int RP, float s,
-                     void* sT_pad, void* T_save, float* part, cudaStream_t st) {
-  if (RP == 64) launch_skinny<64, false>(X, A, M, K, r, s, sT_pad, T_save, part, st);
-  else launch_skinny<128, false>(X, A, M, K, r, s, sT_pad, T_save, part, st);
+                     void* sT_pad, void* T_save, float* part, cudaStream_t st, const Dropout* drop) {
+  const Dropout d = drop ? *drop : Dropout{0, 0, 1.0f, 0};
+  if (RP == 64) launch_skinny<64, false>(X, A, M, K, r, s, sT_pad, T_save, part, d, st);
+  else launch_skinny<128, false>(X, A, M, K, r, s, sT_pad, T_save, part, d, st);
   return skinny_splits(M, K) > 1 ? 2 : 1;
 }
 
 int launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, float s,
                   void* sU_pad, float* part, cudaStream_t st) {
-  if (RP == 64) launch_skinny<64, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, st);
-  else launch_skinny<128, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, st);
+  const Dropout d{0, 0, 1.0f, 0};
+  if (RP == 64) launch_skinny<64, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, d, st);
+  else launch_skinny<128, true>(dY, B, M, N, r, s, sU_pad, nullptr, part, d, st);
   return skinny_splits(M, N) > 1 ? 2 : 1;
 }
 
@@ -255,11 +279,11 @@ int launch_lora_u(const void* dY, const void* B, int M, int N, int r, int RP, fl
 // dA = s U^T X uses P = sU, Q = X;  dB = s dY^T T uses P = dY, Q = T.
 // 8 warps, each 32 x 32 of the tile; operands via ldmatrix.trans.
 // ===========================================================================
-template <int TR, int TC>
+template <int TR, int TC, bool DROPQ>
 __global__ void __launch_bounds__(256)
 k_atb_partial(const __nv_bfloat16* __restrict__ P, int ldp, int Rdim,
               const __nv_bfloat16* __restrict__ Q, int ldq, int Cdim, int M, int rows_per_chunk,
-              float* __restrict__ part, int Rpad, int Cpad) {
+              float* __restrict__ part, int Rpad, int Cpad, Dropout drop) {
   constexpr int MC = 32, STG = 3;
   constexpr int PB = MC * TR * 2, QB = MC * TC * 2;
   constexpr int WC = TC / 32;                       // warps along columns
@@ -309,6 +333,21 @@ k_atb_partial(const __nv_bfloat16* __restrict__ P, int ldp, int Rdim,
     cp_async_commit();
     const uint8_t* ps = sm + (it % STG) * (PB + QB);
     const uint8_t* qs = ps + PB;
+    if (DROPQ) {
+      // LoRA dropout on this stage's rows of Q (the adapter input X)
+      uint8_t* qw = sm + (it % STG) * (PB + QB) + PB;
+      const int mb = mbeg + it * MC;
+      for (int ci = tid; ci < MC * (TC / 8); ci += 256) {
+        const int row = ci / (TC / 8), ch = ci % (TC / 8);
+        const int m = mb + row, cc = c0 + ch * 8;
+        if (m < mend && cc < Cdim) {
+          uint4* q = reinterpret_cast<uint4*>(qw + swzw<TC>(row, ch * 8));
+          *q = dropout8(*q, dropout_keep8(((uint64_t)m * (uint64_t)ldq + (uint64_t)cc) >> 3, drop.seed, drop.thr),
+                        drop.scale);
+        }
+      }
+      __syncthreads();
+    }
 #pragma unroll
     for (int k16 = 0; k16 < MC / 16; ++k16) {
       uint32_t af[2][4];
@@ -378,7 +417,8 @@ int atb_chunks(int tiles, int M) {
 // C[Rdim, Cdim] = s * P^T Q over M rows, bf16 out.  `part` must hold
 // chunks * Rpad * Cpad floats (see atb_workspace_floats).
 void launch_atb(const void* P, int ldp, int Rdim, const void* Q, int ldq, int Cdim, int M, float s,
-                void* out, float* part, int num_sms, cudaStream_t st) {
+                void* out, float* part, int num_sms, cudaStream_t st, const Dropout* dropq) {
+  const Dropout d = dropq ? *dropq : Dropout{0, 0, 1.0f, 0};
   const bool tall = Rdim >= Cdim;                  // choose the tile shape by aspect
   const int TR = tall ? 128 : 64, TC = tall ? 64 : 128;
   const int gr = (Rdim + TR - 1) / TR, gc = (Cdim + TC - 1) / TC;
@@ -388,12 +428,17 @@ void launch_atb(const void* P, int ldp, int Rdim, const void* Q, int ldq, int Cd
   const int nch = (M + rows_per_chunk - 1) / rows_per_chunk;
   const dim3 grid(gr, gc, nch);
   constexpr int smem = 3 * (32 * 128 * 2 + 32 * 64 * 2);
-  if (tall)
-    k_atb_partial<128, 64><<<grid, 256, smem, st>>>((const __nv_bfloat16*)P, ldp, Rdim,
-        (const __nv_bfloat16*)Q, ldq, Cdim, M, rows_per_chunk, part, Rpad, Cpad);
-  else
-    k_atb_partial<64, 128><<<grid, 256, smem, st>>>((const __nv_bfloat16*)P, ldp, Rdim,
-        (const __nv_bfloat16*)Q, ldq, Cdim, M, rows_per_chunk, part, Rpad, Cpad);
+  auto run = [&](auto kern) {
+    kern<<<grid, 256, smem, st>>>((const __nv_bfloat16*)P, ldp, Rdim, (const __nv_bfloat16*)Q, ldq, Cdim,
+                                  M, rows_per_chunk, part, Rpad, Cpad, d);
+  };
+  if (tall) {
+    if (d.on) run(k_atb_partial<128, 64, true>);
+    else run(k_atb_partial<128, 64, false>);
+  } else {
+    if (d.on) run(k_atb_partial<64, 128, true>);
+    else run(k_atb_partial<64, 128, false>);
+  }
   const int64_t total = (int64_t)Rdim * Cdim;
   const int rb = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms * 8);
   k_reduce_partials<<<std::max(rb, 1), 256, 0, st>>>(part, nch, Rpad, Cpad, Rdim, Cdim, s,

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "gemm.h"
 
 namespace qnf4 {
 
@@ -148,7 +149,99 @@ k_qlora_merge(const uint8_t* __restrict__ packed, int N, int K, const float* __r
   }
 }
 
+// Y[M, K] += D * c * (Bm A): the adapter term of dX under LoRA dropout (Bm =
+// s U padded to ldb columns).  Same tiling and tensor-core product as the
+// merge; the epilogue adds into the bf16 Y in place.  The keep bits of a
+// row's 8-column group come from one Philox block, computed once per quad of
+// lanes (lane c of the quad for groups c, c + 4, c + 8, c + 12) and shared by
+// shuffle.
+template <bool DROP>
+__global__ void __launch_bounds__(256)
+k_rank_add(const __nv_bfloat16* __restrict__ Bm, int ldb, const __nv_bfloat16* __restrict__ A, int r,
+           int M, int K, __nv_bfloat16* __restrict__ Y, Dropout drop) {
+  __shared__ __align__(16) uint16_t sA[128][kAPitch];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int k0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile;
+  const int r16 = r < 16 ? 16 : r;
+  for (int i = tid; i < r16 * (kTile / 8); i += 256) {
+    const int j = i / (kTile / 8), ch = i % (kTile / 8);
+    const int k = k0 + ch * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j < r && k < K) v = __ldg(reinterpret_cast<const uint4*>(A + (int64_t)j * K + k));
+    *reinterpret_cast<uint4*>(&sA[j][ch * 8]) = v;
+  }
+  const int ma = m0 + 16 * warp + g, mb = ma + 8;
+  const int ra = min(ma, M - 1), rb = min(mb, M - 1);
+  // keep bits of this lane's four 8-column groups, rows ma and mb
+  uint32_t kb[2][4] = {{0xFFu, 0xFFu, 0xFFu, 0xFFu}, {0xFFu, 0xFFu, 0xFFu, 0xFFu}};
+  if (DROP) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = k0 + 8 * (c + 4 * i);
+        const int m = h ? rb : ra;
+        kb[h][i] = k < K ? dropout_keep8(((uint64_t)m * (uint64_t)K + (uint64_t)k) >> 3, drop.seed, drop.thr) : 0u;
+      }
+  }
+  __syncthreads();
+
+  float acc[16][4];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  for (int kk = 0; kk < r16; kk += 16) {
+    const int j0 = kk + 2 * c, j1 = kk + 8 + 2 * c;
+    const uint32_t a0 = j0 < r ? __ldg(reinterpret_cast<const uint32_t*>(Bm + (int64_t)ra * ldb + j0)) : 0u;
+    const uint32_t a1 = j0 < r ? __ldg(reinterpret_cast<const uint32_t*>(Bm + (int64_t)rb * ldb + j0)) : 0u;
+    const uint32_t a2 = j1 < r ? __ldg(reinterpret_cast<const uint32_t*>(Bm + (int64_t)ra * ldb + j1)) : 0u;
+    const uint32_t a3 = j1 < r ? __ldg(reinterpret_cast<const uint32_t*>(Bm + (int64_t)rb * ldb + j1)) : 0u;
+    const uint32_t row_addr = smem_u32(&sA[kk + (lane & 15)][0]);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      uint32_t b0, b1;
+      ldsm_x2_t(row_addr + t * 16, b0, b1);
+      mma16816_acc(acc[t], a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+  const float cs = DROP ? drop.scale : 1.0f;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    const int k = k0 + 8 * t + 2 * c;
+    // the group's keep bits from lane (g, t % 4) of this quad; columns 2c, 2c + 1
+    uint32_t bits[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t b = DROP ? __shfl_sync(0xffffffffu, kb[h][t >> 2], (lane & ~3) | (t & 3)) : 0xFFu;
+      bits[h] = b >> (2 * c);
+    }
+    if (k >= K) continue;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = h ? mb : ma;
+      if (m >= M) continue;
+      uint32_t* yp = reinterpret_cast<uint32_t*>(Y + (int64_t)m * K + k);
+      const uint32_t y = *yp;
+      const float d0 = (bits[h] & 1u) ? __fmul_rn(cs, acc[t][2 * h]) : 0.0f;
+      const float d1 = (bits[h] & 2u) ? __fmul_rn(cs, acc[t][2 * h + 1]) : 0.0f;
+      *yp = pack_bf16x2(__fadd_rn(bf16_lo(y), d0), __fadd_rn(bf16_hi(y), d1));
+    }
+  }
+}
+
 }  // namespace
+
+void launch_rank_add(const void* Bm, int ldb, const void* A, int r, int M, int K, void* Y,
+                     const Dropout& drop, cudaStream_t st) {
+  const dim3 grid((unsigned)((K + kTile - 1) / kTile), (unsigned)((M + kTile - 1) / kTile));
+  if (drop.on)
+    k_rank_add<true><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Bm, ldb, (const __nv_bfloat16*)A, r, M, K,
+                                           (__nv_bfloat16*)Y, drop);
+  else
+    k_rank_add<false><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Bm, ldb, (const __nv_bfloat16*)A, r, M, K,
+                                            (__nv_bfloat16*)Y, drop);
+}
 
 void launch_merge(const nf4_weight* w, const void* A, const void* B, int r, float s, void* out,
                   cudaStream_t st) {
