@@ -127,25 +127,30 @@ k_qlora_merge(const uint8_t* __restrict__ packed, int N, int K, const float* __r
                            ca[2].x, ca[2].y, ca[2].z, ca[2].w, ca[3].x, ca[3].y, ca[3].z, ca[3].w};
   const uint32_t wb[16] = {cb[0].x, cb[0].y, cb[0].z, cb[0].w, cb[1].x, cb[1].y, cb[1].z, cb[1].w,
                            cb[2].x, cb[2].y, cb[2].z, cb[2].w, cb[3].x, cb[3].y, cb[3].z, cb[3].w};
-  const int na = n0 + 16 * warp + g, nb = na + 8;
+  // the tile is staged in shared memory (the staged A is no longer needed),
+  // then written with 16-byte stores, whole rows per half-warp
+  __syncthreads();
 #pragma unroll
   for (int t = 0; t < 16; ++t) {
     // columns 8t + 2c and 8t + 2c + 1 share code byte 4t + c (byte c of word t)
-    const int k = k0 + 8 * t + 2 * c;
-    if (k >= K) break;
     const int bq = t >> 3;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int n = h ? nb : na;
-      if (n >= N) continue;
       const uint32_t byte = ((h ? wb[t] : wa[t]) >> (8 * c)) & 0xFFu;
       const float a = sc[h][bq];
       const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte >> 4], a)));
       const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_q[byte & 15], a)));
       const float m0 = __fadd_rn(w0, __fmul_rn(s, acc[t][2 * h]));
       const float m1 = __fadd_rn(w1, __fmul_rn(s, acc[t][2 * h + 1]));
-      *reinterpret_cast<uint32_t*>(Wm + (int64_t)n * K + k) = pack_bf16x2(m0, m1);
+      *reinterpret_cast<uint32_t*>(&sA[16 * warp + g + 8 * h][8 * t + 2 * c]) = pack_bf16x2(m0, m1);
     }
+  }
+  __syncthreads();
+  for (int i = tid; i < kTile * (kTile / 8); i += 256) {
+    const int row = i / (kTile / 8), ch = i % (kTile / 8);
+    const int n = n0 + row, k = k0 + ch * 8;
+    if (n < N && k < K)
+      *reinterpret_cast<uint4*>(Wm + (int64_t)n * K + k) = *reinterpret_cast<const uint4*>(&sA[row][ch * 8]);
   }
 }
 
