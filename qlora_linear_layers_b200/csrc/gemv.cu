@@ -25,7 +25,9 @@
 //    8-column operand, one or two tiles).
 //  * Inside each 64-wide NF4 block the contraction order is permuted the same
 //    way for both operands, so that lane (g, c) takes code bytes [8c, 8c+8) of
-//    rows g and g+8 and the activations k in [16c, 16c+16) of its token; the
+//    the tile's rows 2g and 2g+1 (its MMA rows g and g+8: any row order works,
+//    and this one keeps the code loads free of bank conflicts) and the
+//    activations k in [16c, 16c+16) of its token; the
 //    sum is unchanged.
 //  * A code byte (two weights) becomes a bf16 pair through a 256-entry table
 //    of the unscaled NF4 values, replicated per bank so the 32 lanes never
@@ -248,12 +250,16 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
   const uint32_t tsrc = kTableAddr | ((uint32_t)lane * 4);
   const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
   const int NE = p.N + p.r;
+  // MMA row i of a 16-row tile holds weight row 2i (i < 8) or 2(i - 8) + 1:
+  // lane (g, c) reads rows 2g and 2g + 1, whose 128-byte swizzle patterns
+  // (row & 7) put a half-warp's 16 eight-byte reads on all 32 banks.
   // codes: box (j >> 2), logical bytes [(j & 3) * 32 + 8c, +8) of a 128-byte row
   const int cj = (j & 3) * 2 + (c >> 1);
-  const int code_off = (j >> 2) * 8192 + (32 * h + g) * 128 + ((cj ^ g) << 4) + 8 * (c & 1);
+  const int code_off_g = (j >> 2) * 8192 + (32 * h + 2 * g) * 128 + ((cj ^ ((2 * g) & 7)) << 4) + 8 * (c & 1);
+  const int code_off_h = (j >> 2) * 8192 + (32 * h + 2 * g + 1) * 128 + ((cj ^ ((2 * g + 1) & 7)) << 4) + 8 * (c & 1);
   const int xoff = kWBytes + j * 1024 * NT;      // X of block j: 8*NT rows x 128 B
-  // the row whose scale this lane decodes: tile (c & 1), row g + 8 (c >> 1)
-  const int srow = 32 * h + 16 * (c & 1) + g + 8 * (c >> 1);
+  // the row whose scale this lane decodes: tile (c & 1), MMA row g + 8 (c >> 1)
+  const int srow = 32 * h + 16 * (c & 1) + 2 * g + (c >> 1);
 
   float acc[2][NT][4];
 #pragma unroll
@@ -289,7 +295,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int row = 32 * h + 16 * t + g + ((i & 2) ? 8 : 0);
+          const int row = 32 * h + 16 * t + 2 * g + ((i & 2) ? 1 : 0);
           const int tok = nt * 8 + 2 * c + (i & 1);
           if (!ad || (h == 0 && t == 0)) red[row * 16 + tok] = acc[t][nt][i];
           acc[t][nt][i] = 0.f;
@@ -347,14 +353,21 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     if (b < p.nb && (nf4 || h == 0)) {
       uint32_t xw[NT][8];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) lds_row16(sb + xoff, nt * 8 + g, c, xw[nt]);
+      for (int nt = 0; nt < NT; ++nt) {
+        if (nt * 8 + g < p.M) {
+          lds_row16(sb + xoff, nt * 8 + g, c, xw[nt]);
+        } else {                                 // token rows past M are zero
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xw[nt][i] = 0u;
+        }
+      }
       if (nf4) {
         // ---- 32 NF4 rows x one block
         uint2 wg[2], wh[2];
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          wg[t] = *reinterpret_cast<const uint2*>(sb + code_off + t * 16 * 128);
-          wh[t] = *reinterpret_cast<const uint2*>(sb + code_off + t * 16 * 128 + 8 * 128);
+          wg[t] = *reinterpret_cast<const uint2*>(sb + code_off_g + t * 16 * 128);
+          wh[t] = *reinterpret_cast<const uint2*>(sb + code_off_h + t * 16 * 128);
         }
         float cb[2][NT][4];
 #pragma unroll
@@ -398,8 +411,8 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       } else {
         // ---- 16 bf16 rows of A x one block: T[m, j] = sum_k X[m, k] A[j, k]
         uint32_t gw4[8], hw4[8];
-        lds_row16(sb + j * 2048, g, c, gw4);       // rows past r were zero-filled
-        lds_row16(sb + j * 2048, g + 8, c, hw4);
+        lds_row16(sb + j * 2048, 2 * g, c, gw4);   // rows past r were zero-filled
+        lds_row16(sb + j * 2048, 2 * g + 1, c, hw4);
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[s]);
 #pragma unroll
