@@ -376,6 +376,24 @@ int qlora_linear_fwd_noalloc(const nf4_weight* w, const void* X, int64_t M,
  */
 int qlora_check_status(qlora_stream_t stream);
 
+/*
+ * Failure detection.  Every pipeline wait in the library's kernels (on a
+ * TMA stage, a tensor-core commit, the partner SM of a pair) gives up after
+ * a wall-time limit: the kernel records QLORA_ERR_TIMEOUT in the status
+ * word, lets the copies it issued land (bounded too), releases its tensor
+ * memory and returns, so the context stays usable.
+ *   qlora_set_wait_limit: the limit for the current device, in ns (0 = the
+ *     default 1 s; otherwise 1 ms .. 60 s, else QLORA_ERR_INVALID_ARG).
+ *     Synchronous; do not change it while the library's kernels run.
+ *   qlora_test_withhold_first_fill: a test switch (default off).  While on,
+ *     the decode kernel's first CTA leaves its first pipeline stage
+ *     unfilled, so that its waits run out and the call reports
+ *     QLORA_ERR_TIMEOUT -- a wait that nothing satisfies, with no fault.
+ * Both return QLORA_OK or QLORA_ERR_CUDA / QLORA_ERR_UNSUPPORTED.
+ */
+int qlora_set_wait_limit(uint64_t ns);
+int qlora_test_withhold_first_fill(int on);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

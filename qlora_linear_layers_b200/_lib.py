@@ -92,6 +92,8 @@ SIGNATURES = {
     "qlora_linear_fwd_noalloc": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,
                                         _vp, _vp, _vp]),
     "qlora_check_status": (_i32, [_vp]),
+    "qlora_set_wait_limit": (_i32, [C.c_uint64]),
+    "qlora_test_withhold_first_fill": (_i32, [_i32]),
 }
 
 _lib = None

@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <cuda_runtime.h>
@@ -14,8 +15,9 @@
 
 namespace qnf4 {
 
-// One status word per device (each device context has its own copy).
-static __device__ int g_status = 0;
+// One state block per device (each device context has its own copy): the
+// status word, the test switch and the wait limit.
+static __device__ DevState g_state = {0, 0, kWaitLimitNs};
 
 namespace {
 
@@ -48,8 +50,8 @@ int current_device(DeviceInfo** info) {
     d.major = p.major;
     d.minor = p.minor;
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_CUDA; }
-    d.status = static_cast<int*>(ptr);
+    if (cudaGetSymbolAddress(&ptr, g_state) != cudaSuccess) { cudaGetLastError(); return QLORA_ERR_CUDA; }
+    d.status = &static_cast<DevState*>(ptr)->status;
     d.ready = true;
   }
   if (d.major != 10) return QLORA_ERR_UNSUPPORTED;   // sm_100 family only
@@ -567,6 +569,31 @@ int qlora_linear_bwd_dropout(const nf4_weight* w, const void* X, const void* dY,
   const int st = make_dropout(dropout, &dr);
   if (st) return st;
   return bwd_impl(w, X, dY, M, A, B, r, alpha, &dr, T, dX, dA, dB, ws, ws_bytes, stream);
+}
+
+// Write one field of the current device's state block (synchronous).
+static int write_state_field(size_t offset, const void* src, size_t bytes) {
+  DeviceInfo* d = nullptr;
+  int st = current_device(&d);
+  if (st) return st;
+  if (cudaMemcpy(reinterpret_cast<uint8_t*>(d->status) + offset, src, bytes, cudaMemcpyHostToDevice) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+int qlora_set_wait_limit(uint64_t ns) {
+  if (ns == 0) ns = kWaitLimitNs;
+  if (ns < 1000000ull || ns > 60000000000ull) return QLORA_ERR_INVALID_ARG;
+  const unsigned long long v = ns;
+  return write_state_field(offsetof(DevState, wait_limit_ns), &v, sizeof(v));
+}
+
+int qlora_test_withhold_first_fill(int on) {
+  const int v = on ? 1 : 0;
+  return write_state_field(offsetof(DevState, withhold_first_fill), &v, sizeof(v));
 }
 
 int qlora_check_status(qlora_stream_t stream) {

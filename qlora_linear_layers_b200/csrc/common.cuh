@@ -11,12 +11,24 @@
 namespace qnf4 {
 
 // ---------------------------------------------------------------------------
-// Sticky device status word (one per device, defined in capi.cu).  Every
-// kernel receives its address; the first error is kept (atomicCAS from 0);
-// qlora_check_status() reads and clears it.
+// Per-device state block (defined in capi.cu): the sticky status word first,
+// then the wait limit every bounded wait uses and one test switch.  Every
+// kernel receives the address of the status word (the block's start); the
+// first error is kept (atomicCAS from 0); qlora_check_status() reads and
+// clears it.
 // ---------------------------------------------------------------------------
+struct DevState {
+  int status;
+  int withhold_first_fill;       // test switch: the decode kernel's CTA 0 skips its first stage fill
+  unsigned long long wait_limit_ns;
+};
+
 __device__ __forceinline__ void set_status(int* st, int code) {
   atomicCAS(st, 0, code);
+}
+
+__device__ __forceinline__ uint64_t wait_limit_ns(const int* st) {
+  return *reinterpret_cast<const volatile unsigned long long*>(&reinterpret_cast<const DevState*>(st)->wait_limit_ns);
 }
 
 int* device_status_ptr();   // host: address of the status word on the current device
@@ -64,8 +76,9 @@ struct CodeTables {
 // QLORA_QUANT_FP4 (anything else: NF4).
 const CodeTables& host_tables(int quant_type = QLORA_QUANT_NF4);
 
-// Every pipeline wait gives up after this much wall time (ns), far above any
-// legitimate wait (the longest stage hand-off is microseconds).
+// Every pipeline wait gives up after the device state's wait limit (1 s by
+// default: far above any legitimate wait, the longest stage hand-off is
+// microseconds; qlora_set_wait_limit changes it).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -193,17 +206,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false (and records QLORA_ERR_TIMEOUT) if the phase
-// does not complete within kWaitLimitNs.  `abort` is a CTA-shared flag: once
+// does not complete within the wait limit.  `abort` is a CTA-shared flag: once
 // any waiter gives up, the others stop waiting too.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort, int* st) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns(st);
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (globaltimer_ns() - t0 > limit) break;
     }
   }
   *abort = 1;
@@ -355,11 +369,12 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
                                                   volatile int* abort, int* st) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns(st);
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (globaltimer_ns() - t0 > limit) break;
     }
   }
   *abort = 1;

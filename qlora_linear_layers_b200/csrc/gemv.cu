@@ -139,10 +139,11 @@ __device__ __forceinline__ void consumer_sync() {
 }
 
 // Wait for a stage's copy after an abort, bounded, ignoring the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const int* st) {
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns(st);
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    if (globaltimer_ns() - t0 > limit) break;
 }
 
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
@@ -216,11 +217,19 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       uint32_t k = 0;
       bool ok = true;
       int rgp = (int)(u0 / p.spr), st = (int)(u0 - (int64_t)rgp * p.spr);
+      // test switch: CTA 0 leaves its first stage unfilled, so that its
+      // consumers' bounded waits run out (QLORA_ERR_TIMEOUT)
+      const bool withhold = blockIdx.x == 0 &&
+                            reinterpret_cast<const volatile DevState*>(p.status)->withhold_first_fill != 0;
       for (int64_t u = u0; u < u1; ++u, ++k) {
         const int s = (int)(k % kStages);
         if (!(ok = mbar_wait(&S.empty[s], ((k / kStages) & 1) ^ 1, abort, p.status))) break;
         const int b = st * kBlk;
         uint8_t* dst = stage_ptr(s);
+        if (withhold && k == 0) {
+          if (++st == p.spr) { st = 0; ++rgp; }
+          continue;
+        }
         mbar_arrive_expect_tx(&S.full[s], kTx);
         if (rgp < p.nat) {
           tma_load_3d(dst, &tm_a, &S.full[s], 0, rgp * kARows, b);
@@ -235,7 +244,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       if (!ok) {
         // a wait gave up: let the copies in flight land before the CTA exits
         for (uint32_t i = (k > (uint32_t)kStages ? k - kStages : 0); i < k; ++i)
-          drain_wait(&S.full[i % kStages], (i / kStages) & 1);
+          drain_wait(&S.full[i % kStages], (i / kStages) & 1, p.status);
       }
     }
     return;

@@ -159,3 +159,8 @@ def test_host_mean_from_histogram_matches_oracle(lib):
     h[3] = -1
     assert lib.qlora_dq_mean_from_hist(h.ctypes.data_as(C.POINTER(C.c_int64)), 1, C.byref(mean)) == \
         _lib.QLORA_ERR_INVALID_ARG
+
+
+def test_wait_limit_range_checked_on_the_host(lib):
+    assert lib.qlora_set_wait_limit(1000) == _lib.QLORA_ERR_INVALID_ARG            # below 1 ms
+    assert lib.qlora_set_wait_limit(61 * 10 ** 9) == _lib.QLORA_ERR_INVALID_ARG    # above 60 s
