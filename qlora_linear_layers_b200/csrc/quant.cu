@@ -17,10 +17,12 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise: one thread owns one 64-weight block (eight 16-byte bf16 loads or
-// sixteen fp32 ones, a 32-byte code store and its absmax), so the block max,
-// the reciprocal and the stores cost one thread's work per 64 weights, and a
-// warp's 32 blocks are contiguous.  absmax is an integer max over |w| bit
+// Quantise: one thread owns one 64-weight block at a time (eight 16-byte
+// bf16 loads or sixteen fp32 ones, a 32-byte code store and its absmax), so
+// the block max, the reciprocal and the stores cost one thread's work per 64
+// weights, and a warp's 32 blocks are contiguous.  A persistent grid (two
+// CTAs per SM) walks the blocks; each thread loads its next block's words
+// before it computes the current block's codes.  absmax is an integer max over |w| bit
 // patterns (exact; NaN/Inf show up as >= 0x7f800000).
 //
 // Code of x = RN32(w / a):  x' = RN32(w * rcp(a)) with the hardware reciprocal
@@ -81,10 +83,11 @@ template <> struct BlockWords<__nv_bfloat16> {
     return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
   }
   __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
-    uint32_t m = 0;
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j = 0; j < kWords; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
-    return max(m << 16, m & 0xFFFF0000u);
+    for (int j = 0; j < kWords; ++j) m[j & 3] = __vmaxu2(m[j & 3], w[j] & 0x7FFF7FFFu);
+    const uint32_t mm = __vmaxu2(__vmaxu2(m[0], m[1]), __vmaxu2(m[2], m[3]));
+    return max(mm << 16, mm & 0xFFFF0000u);
   }
 };
 template <> struct BlockWords<float> {
@@ -125,7 +128,7 @@ __device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float
 }
 
 template <typename T, bool MONO, bool HIST>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
            float* __restrict__ absmax, unsigned long long* __restrict__ hist, CodeTables tb,
            int* status) {
@@ -143,18 +146,29 @@ k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packe
   const uint32_t lane_base = smem_u32(s_bk) + (uint32_t)lane * 8u;
   constexpr int kWords = BlockWords<T>::kWords;
   bool bad = false;
-  // warp-uniform loop (the histogram's match/reduce need whole warps)
+  // warp-uniform loop (the histogram's match/reduce need whole warps); the
+  // next block's words are loaded before this block's codes are computed
   const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  for (int64_t base = first; base < nblk; base += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t gstride = (int64_t)gridDim.x * blockDim.x;
+  uint32_t wn[kWords];
+  auto load_words = [&](int64_t base_) {
+    const int64_t b = base_ + lane;
+    const bool v_ = b < nblk;
+    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * (v_ ? b : 0);
+#pragma unroll
+    for (int k = 0; k < kWords / 4; ++k) {
+      const uint4 v = v_ ? __ldcs(src + k) : make_uint4(0u, 0u, 0u, 0u);
+      wn[4 * k] = v.x; wn[4 * k + 1] = v.y; wn[4 * k + 2] = v.z; wn[4 * k + 3] = v.w;
+    }
+  };
+  if (first < nblk) load_words(first);
+  for (int64_t base = first; base < nblk; base += gstride) {
     const int64_t blk = base + lane;
     const bool valid = blk < nblk;
     uint32_t w[kWords];
-    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * (valid ? blk : 0);
 #pragma unroll
-    for (int k = 0; k < kWords / 4; ++k) {
-      const uint4 v = valid ? __ldcs(src + k) : make_uint4(0u, 0u, 0u, 0u);
-      w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
-    }
+    for (int k = 0; k < kWords; ++k) w[k] = wn[k];
+    if (base + gstride < nblk) load_words(base + gstride);
     uint32_t m = BlockWords<T>::absmax_bits(w);
     if (m >= 0x7F800000u) { bad = true; m = 0; }
     const float a = __uint_as_float(m);
@@ -207,8 +221,11 @@ static void launch_quantize_t(const void* W, int64_t nblk, uint8_t* packed, floa
                               cudaStream_t s) {
   constexpr int kThreads = 256;
   // one block per thread: other CTAs' loads cover each block's compute
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nblk + kThreads - 1) / kThreads,
-                                                                 (int64_t)1 << 30));
+                                                                 (int64_t)sms * 2));
   if (hist)
     k_quantize<T, MONO, true><<<blocks, kThreads, 0, s>>>(W, nblk, packed, absmax, hist, tb, status);
   else
