@@ -68,6 +68,14 @@ typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
  *     and is never produced by quantisation. */
 typedef enum { QLORA_QUANT_NF4 = 0, QLORA_QUANT_FP4 = 1 } qlora_quant_type;
 
+/* Formats of the 8-bit block-scale codes (nf4_weight.double_quant):
+ *   QLORA_DQ_INT8: symmetric int8, c = round-half-even(RN32(RN32(d / s_g) * 127))
+ *   QLORA_DQ_FP8:  the E4M3 8-bit float (sign, 4 exponent bits with bias 7,
+ *                  3 mantissa bits), c = E4M3(256 * RN32(d / s_g)) rounded to
+ *                  nearest with ties to the even code (the sign of a zero
+ *                  result is kept); decoded exactly as e4m3(c) / 256. */
+typedef enum { QLORA_DQ_NONE = 0, QLORA_DQ_INT8 = 1, QLORA_DQ_FP8 = 2 } qlora_dq_type;
+
 /* Bytes of the double-quantisation exponent histogram: 256 int64 bins; bin e
  * holds the sum of the 24-bit significands of the absmax values whose fp32
  * exponent field is e (bin 255 unused).  Histograms of disjoint parts of a
@@ -115,7 +123,9 @@ typedef struct {
  *
  * Dequantised value of element i in block b (code c, table q of quant_type):
  *   a^ = absmax[b]                                              (no DQ)
- *   a^ = RN32(RN32(RN32(qabsmax[b]/127) * dq_scale[b/256]) + dq_mean) (DQ)
+ *   a^ = RN32(RN32(v(qabsmax[b]) * dq_scale[b/256]) + dq_mean)  (DQ)
+ *   v(c) = RN32(c / 127) for int8 codes (double_quant 1), e4m3(c) / 256 for
+ *   8-bit float codes (double_quant 2; c is the E4M3 byte)
  *   w' = RNbf16(RN32(q[c] * a^))
  * quant_type is QLORA_QUANT_NF4 (0) or QLORA_QUANT_FP4 (1); a zero-filled
  * struct is NF4.
@@ -125,7 +135,7 @@ typedef struct {
   int64_t rows;
   int64_t cols;
   int32_t blocksize;      /* must be 64  */
-  int32_t double_quant;   /* 0 or 1      */
+  int32_t double_quant;   /* 0: none, 1 (QLORA_DQ_INT8) or 2 (QLORA_DQ_FP8) */
   const float* absmax;
   const int8_t* qabsmax;
   const float* dq_scale;
@@ -249,6 +259,13 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
 int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
                              int64_t n_total, int dq_blocksize, int8_t* qabsmax,
                              float* dq_scale, float* dq_mean, qlora_stream_t stream);
+
+/* The same with the code format chosen: dq_type QLORA_DQ_INT8 (as above) or
+ * QLORA_DQ_FP8 (see qlora_dq_type); the weight's double_quant field must
+ * then name the same format. */
+int qlora_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
+                               int64_t n_total, int dq_blocksize, int dq_type, int8_t* qabsmax,
+                               float* dq_scale, float* dq_mean, qlora_stream_t stream);
 
 /*
  * Dequantise to bf16 ([QE] worked example step 4; "That is NF4": every

@@ -46,6 +46,9 @@ from .nf4 import (  # noqa: F401
     dq_mean,
     double_quantize,
     dq_absmax,
+    e4m3_values,
+    e4m3_encode,
+    e4m3_decode,
     dequantize,
     round_bf16,
     stored_bits_per_param,

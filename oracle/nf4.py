@@ -261,7 +261,43 @@ def dq_mean(absmax: np.ndarray) -> np.float32:
     return np.float32(s / a.size)                    # fp64 divide, then RN32
 
 
-def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE):
+def e4m3_values() -> np.ndarray:
+    """The 127 non-negative finite values of the 8-bit float E4M3 (sign bit,
+    4 exponent bits with bias 7, 3 mantissa bits; exponent field 15 with
+    mantissa 7 is NaN), by code 0..126, exact in fp64:
+      e == 0:  m / 8 * 2^-6           (subnormal)
+      e >  0:  (1 + m / 8) * 2^(e - 7)"""
+    out = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        out.append((m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(out, dtype=np.float64)
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """E4M3 code (uint8) of each fp32 value: the nearest finite value, a tie
+    to the even code, magnitudes above 448 saturated to 448; the sign bit is
+    kept, so a negative value that rounds to zero is -0 (code 0x80)."""
+    v = e4m3_values()
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), v[-1])
+    hi = np.clip(np.searchsorted(v, a, side="left"), 0, v.size - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - v[lo], v[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    """fp64 value of E4M3 codes (NaN codes 0x7F / 0xFF give NaN)."""
+    c = np.asarray(code, dtype=np.uint8)
+    mag = c & 0x7F
+    v = np.append(e4m3_values(), np.nan)[mag]
+    return np.where(c & 0x80, -v, v)
+
+
+def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE, fmt: str = "int8"):
     """8-bit quantisation of the block scales in groups of 256.
 
     Page "QLoRA Explained", section "Shrink the scale factors too": each scale
@@ -276,7 +312,15 @@ def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE):
       s_g == 0  ->  c = 0
 
     Returns (qabsmax int8[n], dq_scale fp32[ceil(n/256)], mu fp32).
+
+    fmt = "fp8": the 8-bit float variant (the pages name no 8-bit format; the
+    original method's second level is an 8-bit float).  Reading: the same d,
+    s_g and t = RN32(d / s_g), then the E4M3 code of 256 * t (exact scaling;
+    E4M3's largest value 448 is never reached), round to nearest, ties to the
+    even code; the code bytes are returned in the int8 array.
     """
+    if fmt not in ("int8", "fp8"):
+        raise ValueError("fmt must be int8 or fp8")
     a = np.asarray(absmax, dtype=np.float32).reshape(-1)
     mu = dq_mean(a)
     d = (a - mu).astype(np.float32)                              # RN32(a - mu)
@@ -290,6 +334,10 @@ def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE):
         if sg == 0:
             continue
         t = (dg / sg).astype(np.float32)                         # RN32(d / s_g)
+        if fmt == "fp8":
+            u = (t * np.float32(256)).astype(np.float32)         # exact
+            q[g * dq_blocksize:(g + 1) * dq_blocksize] = e4m3_encode(u).view(np.int8)
+            continue
         t = (t * np.float32(127)).astype(np.float32)             # RN32(. * 127)
         c = np.rint(t)                                           # half to even
         q[g * dq_blocksize:(g + 1) * dq_blocksize] = np.clip(c, -127, 127).astype(np.int8)
@@ -297,11 +345,16 @@ def double_quantize(absmax: np.ndarray, dq_blocksize: int = DQ_BLOCKSIZE):
 
 
 def dq_absmax(qabsmax: np.ndarray, dq_scale: np.ndarray, mu,
-              dq_blocksize: int = DQ_BLOCKSIZE) -> np.ndarray:
-    """Recovered block scale a^ = RN32( RN32( RN32(c / 127) * s_g ) + mu )."""
-    c = np.asarray(qabsmax, dtype=np.int8).astype(np.float32)
-    s = np.repeat(np.asarray(dq_scale, dtype=np.float32), dq_blocksize)[: c.size]
-    t = (c / np.float32(127)).astype(np.float32)                 # RN32(c / 127)
+              dq_blocksize: int = DQ_BLOCKSIZE, fmt: str = "int8") -> np.ndarray:
+    """Recovered block scale a^ = RN32( RN32( RN32(c / 127) * s_g ) + mu ),
+    or with fmt = "fp8" RN32( RN32( (e4m3(c) / 256) * s_g ) + mu ) (the
+    division by 256 is exact)."""
+    s = np.repeat(np.asarray(dq_scale, dtype=np.float32), dq_blocksize)[: np.asarray(qabsmax).size]
+    if fmt == "fp8":
+        t = (e4m3_decode(np.asarray(qabsmax).view(np.uint8)) / 256.0).astype(np.float32)
+    else:
+        c = np.asarray(qabsmax, dtype=np.int8).astype(np.float32)
+        t = (c / np.float32(127)).astype(np.float32)             # RN32(c / 127)
     t = (t * s).astype(np.float32)                               # RN32(. * s_g)
     return (t + np.float32(mu)).astype(np.float32)               # RN32(. + mu)
 

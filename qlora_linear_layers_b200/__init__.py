@@ -48,13 +48,13 @@ class NF4Tensor:
     qabsmax: torch.Tensor | None    # int8 [rows*cols/64]
     dq_scale: torch.Tensor | None   # fp32 [ceil(n_absmax/256)]
     dq_mean: torch.Tensor | None    # fp32 [1]
-    double_quant: bool = True
+    double_quant: int = 1           # 0 none, 1 int8 codes, 2 E4M3 codes (True = 1)
     quant_type: int = _lib.QLORA_QUANT_NF4
 
     def c_struct(self) -> _lib.NF4Weight:
         return _lib.NF4Weight(
             packed=_ptr(self.packed), rows=self.rows, cols=self.cols, blocksize=BLOCKSIZE,
-            double_quant=1 if self.double_quant else 0,
+            double_quant=int(self.double_quant),
             absmax=_ptr(self.absmax), qabsmax=_ptr(self.qabsmax), dq_scale=_ptr(self.dq_scale),
             dq_mean=_ptr(self.dq_mean), dq_blocksize=DQ_BLOCKSIZE, quant_type=self.quant_type)
 
@@ -99,14 +99,16 @@ def qlora_quantize_4bit(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Ten
 
 def nf4_double_quantize_hist(absmax: torch.Tensor, dq_hist: torch.Tensor, n_total: int,
                              qabsmax: torch.Tensor, dq_scale: torch.Tensor, dq_mean: torch.Tensor,
-                             stream=None):
+                             stream=None, dq_type: int = _lib.QLORA_DQ_INT8):
     """Second double-quantisation pass from a complete histogram over n_total
-    absmax values (summed over shards when the weight is sharded)."""
+    absmax values (summed over shards when the weight is sharded); dq_type
+    picks int8 or E4M3 codes."""
     _need_cuda(absmax, dq_hist, qabsmax, dq_scale, dq_mean)
-    _lib.check(_lib.load().nf4_double_quantize_hist(_ptr(absmax), absmax.numel(), _ptr(dq_hist),
-                                                    int(n_total), DQ_BLOCKSIZE, _ptr(qabsmax),
-                                                    _ptr(dq_scale), _ptr(dq_mean), _stream(stream)),
-               "nf4_double_quantize_hist")
+    _lib.check(_lib.load().qlora_double_quantize_hist(_ptr(absmax), absmax.numel(), _ptr(dq_hist),
+                                                      int(n_total), DQ_BLOCKSIZE, int(dq_type),
+                                                      _ptr(qabsmax), _ptr(dq_scale), _ptr(dq_mean),
+                                                      _stream(stream)),
+               "qlora_double_quantize_hist")
 
 
 def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
@@ -226,7 +228,7 @@ def code_thresholds(quant_type: int = _lib.QLORA_QUANT_NF4) -> list[float]:
 # Conveniences
 # ---------------------------------------------------------------------------
 
-def empty_quantized(rows: int, cols: int, device, double_quant: bool = True,
+def empty_quantized(rows: int, cols: int, device, double_quant: int = 1,
                     quant_type: int = _lib.QLORA_QUANT_NF4) -> NF4Tensor:
     """Buffers of a quantised [rows, cols] weight (absmax is kept either way:
     the quantise pass writes it)."""
@@ -234,7 +236,7 @@ def empty_quantized(rows: int, cols: int, device, double_quant: bool = True,
     na = n // BLOCKSIZE
     t = NF4Tensor(torch.empty(n // 2, dtype=torch.uint8, device=device), rows, cols,
                   torch.empty(na, dtype=torch.float32, device=device), None, None, None,
-                  double_quant, quant_type)
+                  int(double_quant), quant_type)
     if double_quant:
         t.qabsmax = torch.empty(na, dtype=torch.int8, device=device)
         t.dq_scale = torch.empty((na + DQ_BLOCKSIZE - 1) // DQ_BLOCKSIZE, dtype=torch.float32,
@@ -243,19 +245,21 @@ def empty_quantized(rows: int, cols: int, device, double_quant: bool = True,
     return t
 
 
-def quantize(W: torch.Tensor, double_quant: bool = True, quant_type: int = _lib.QLORA_QUANT_NF4,
+def quantize(W: torch.Tensor, double_quant: int = 1, quant_type: int = _lib.QLORA_QUANT_NF4,
              stream=None) -> NF4Tensor:
-    """Quantise W; with double quantisation the histogram of the mean is built
-    in the quantise pass and one more pass writes the 8-bit scales."""
+    """Quantise W.  double_quant: 0 (or False) keeps fp32 block scales, 1 (or
+    True) int8 codes, 2 E4M3 codes; the mean's histogram is built in the
+    quantise pass and one more pass writes the 8-bit scales."""
     rows, cols = W.shape
-    q = empty_quantized(rows, cols, W.device, double_quant, quant_type)
-    if not double_quant:
+    dq = int(double_quant)
+    q = empty_quantized(rows, cols, W.device, dq, quant_type)
+    if not dq:
         qlora_quantize_4bit(W, q.packed, q.absmax, quant_type, None, stream)
         return q
     hist = torch.empty(256, dtype=torch.int64, device=W.device)
     qlora_quantize_4bit(W, q.packed, q.absmax, quant_type, hist, stream)
     nf4_double_quantize_hist(q.absmax, hist, q.absmax.numel(), q.qabsmax, q.dq_scale, q.dq_mean,
-                             stream)
+                             stream, dq_type=dq)
     return q
 
 

@@ -29,6 +29,9 @@ QLORA_BF16 = 1
 QLORA_QUANT_NF4 = 0
 QLORA_QUANT_FP4 = 1
 QLORA_DQ_HIST_BYTES = 2048
+QLORA_DQ_NONE = 0
+QLORA_DQ_INT8 = 1
+QLORA_DQ_FP8 = 2
 
 QLORA_OP_DOUBLE_QUANT = 0
 QLORA_OP_FWD = 1
@@ -79,6 +82,7 @@ SIGNATURES = {
     "qlora_quantize_4bit": (_i32, [_vp, _i32, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
     "nf4_double_quantize": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nf4_double_quantize_hist": (_i32, [_vp, _i64, _vp, _i64, _i32, _vp, _vp, _vp, _vp]),
+    "qlora_double_quantize_hist": (_i32, [_vp, _i64, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]),
     "nf4_dequantize": (_i32, [C.POINTER(NF4Weight), _vp, _vp]),
     "qlora_merge": (_i32, [C.POINTER(NF4Weight), _vp, _vp, _i32, _f32, _vp, _vp]),
     "qlora_linear_fwd": (_i32, [C.POINTER(NF4Weight), _vp, _i64, _vp, _vp, _i32, _f32,

@@ -121,6 +121,7 @@ int check_weight(const nf4_weight* w) {
   if (w->quant_type != QLORA_QUANT_NF4 && w->quant_type != QLORA_QUANT_FP4) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 64 || w->cols % 64) return QLORA_ERR_SHAPE;
   if (!aligned16(w->packed)) return QLORA_ERR_ALIGN;
+  if (w->double_quant < 0 || w->double_quant > 2) return QLORA_ERR_INVALID_ARG;
   if (w->double_quant) {
     if (w->dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
     if (!w->qabsmax || !w->dq_scale || !w->dq_mean) return QLORA_ERR_INVALID_ARG;
@@ -345,7 +346,15 @@ int nf4_double_quantize(const float* absmax, int64_t n_absmax, int dq_blocksize,
 int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
                              int64_t n_total, int dq_blocksize, int8_t* qabsmax, float* dq_scale,
                              float* dq_mean, qlora_stream_t stream) {
+  return qlora_double_quantize_hist(absmax, n_absmax, dq_hist, n_total, dq_blocksize, QLORA_DQ_INT8,
+                                    qabsmax, dq_scale, dq_mean, stream);
+}
+
+int qlora_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_t* dq_hist,
+                               int64_t n_total, int dq_blocksize, int dq_type, int8_t* qabsmax,
+                               float* dq_scale, float* dq_mean, qlora_stream_t stream) {
   if (!absmax || !dq_hist || !qabsmax || !dq_scale || !dq_mean) return QLORA_ERR_INVALID_ARG;
+  if (dq_type != QLORA_DQ_INT8 && dq_type != QLORA_DQ_FP8) return QLORA_ERR_INVALID_ARG;
   if (dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
   if (n_absmax < 1 || n_total < n_absmax || n_total > ((int64_t)1 << 39)) return QLORA_ERR_SHAPE;
   if (!aligned16(absmax) || !aligned16(dq_hist) || !aligned16(qabsmax) || !aligned16(dq_scale) ||
@@ -357,7 +366,7 @@ int nf4_double_quantize_hist(const float* absmax, int64_t n_absmax, const int64_
   const int n = launch_double_quantize_from_hist(absmax, n_absmax,
                                                  reinterpret_cast<const unsigned long long*>(dq_hist),
                                                  n_total, qabsmax, dq_scale, dq_mean,
-                                                 (cudaStream_t)stream, d->sms);
+                                                 (cudaStream_t)stream, d->sms, dq_type);
   st = launch_status();
   if (!st) count_launches(n);
   return st;

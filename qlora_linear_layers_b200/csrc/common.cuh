@@ -88,6 +88,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// Value of an 8-bit block-scale code, as the entry idx = c + 128 of a 256-entry
+// table (c the stored byte read as int8):
+//   dq_type 1 (int8):  RN32(c / 127)
+//   dq_type 2 (E4M3 byte b = idx ^ 0x80):  e4m3(b) / 256 (exact)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float dq_code_value(int idx, int dq_type) {
+  if (dq_type == 2) {
+    const uint32_t b = (uint32_t)idx ^ 0x80u;
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    // subnormal m * 2^-9; normal (1 + m/8) * 2^(e - 7): exponent field e + 120
+    float v = e == 0 ? (float)m * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    if (e == 15u && m == 7u) v = __int_as_float(0x7fc00000);     // the NaN code (never written)
+    v = v * 0x1p-8f;
+    return (b & 0x80u) ? -v : v;
+  }
+  return __fdiv_rn((float)(idx - 128), 127.0f);
+}
+
+// ---------------------------------------------------------------------------
 // LoRA dropout mask: Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel
 // Random Numbers: As Easy as 1, 2, 3", SC 2011) with key (seed, 0) and
 // counter (e / 8, 0, 0, 0) for element e = m * K + k of the adapter input;

@@ -109,7 +109,7 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     mbar_fence_init();
   }
   for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    S.inv127[i] = __fdiv_rn((float)(i - 128), 127.0f);   // entry c + 128: any int8 c
+    S.inv127[i] = dq_code_value(i, p.double_quant);     // entry c + 128: any code byte
   if (warp == 1) {
     tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
     tmem_relinquish_pair();

@@ -108,6 +108,7 @@ struct GemvArgs {
   int64_t U;                  // units: (nat + nrg) * spr
   int P;                      // ranges (CTAs): min(148, U)
   uint32_t smem_base;         // shared-window address of dynamic shared memory
+  int dq_type;                // 1: int8 block-scale codes, 2: E4M3
   float q[16];
 };
 
@@ -192,7 +193,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       tbl[e * 64 + l] = pack_bf16x2(p.q[e >> 4], p.q[e & 15]);   // element 2j (high nibble) low half
     }
   }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) S.inv127[i] = __fdiv_rn((float)(i - 128), 127.0f);   // entry c + 128: any int8 c
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) S.inv127[i] = dq_code_value(i, p.dq_type);   // entry c + 128: any code byte
   if (threadIdx.x == 0) {
     S.abort = 0;
     for (int i = 0; i < kStages; ++i) {
@@ -589,6 +590,7 @@ int launch_qlora_gemv(const nf4_weight* w, const void* X, int M, const void* A, 
   GemvArgs a{};
   a.status = status;
   a.absmax = w->absmax; a.qabsmax = w->qabsmax;
+  a.dq_type = w->double_quant;
   a.dq_scale = w->dq_scale; a.dq_mean = w->dq_mean;
   a.part = part;
   a.M = M; a.N = (int)w->rows; a.K = (int)w->cols; a.r = r;

@@ -25,7 +25,7 @@ int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, floa
 // number of launches.
 int launch_double_quantize_from_hist(const float* absmax, int64_t n, const unsigned long long* hist,
                                      int64_t n_total, int8_t* qabsmax, float* dq_scale, float* dq_mean,
-                                     cudaStream_t s, int num_sms);
+                                     cudaStream_t s, int num_sms, int dq_type);
 
 void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_sms);
 

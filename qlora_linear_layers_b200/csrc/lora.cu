@@ -480,8 +480,7 @@ k_dequant_t(const uint8_t* __restrict__ packed, int N, int K, int dq,
       const int64_t blk = e >> 6;
       float a;
       if (dq) {
-        const float c = (float)qabsmax[blk];
-        a = __fadd_rn(__fmul_rn(__fdiv_rn(c, 127.0f), dq_scale[blk >> 8]), dq_mean[0]);
+        a = __fadd_rn(__fmul_rn(dq_code_value((int)qabsmax[blk] + 128, dq), dq_scale[blk >> 8]), dq_mean[0]);
       } else {
         a = absmax[blk];
       }

@@ -56,7 +56,7 @@ k_qlora_merge(const uint8_t* __restrict__ packed, int N, int K, const float* __r
               const int8_t* __restrict__ qabsmax, const float* __restrict__ dq_scale,
               const float* __restrict__ dq_mean, const __nv_bfloat16* __restrict__ A,
               const __nv_bfloat16* __restrict__ B, int r, float s, __nv_bfloat16* __restrict__ Wm,
-              CodeTables tb) {
+              CodeTables tb, int dq_type) {
   __shared__ __align__(16) uint16_t sA[128][kAPitch];    // rows j < r16 of A, the tile's columns
   __shared__ float s_q[16];
   __shared__ float s_inv127[256];
@@ -65,7 +65,7 @@ k_qlora_merge(const uint8_t* __restrict__ packed, int N, int K, const float* __r
   const int k0 = blockIdx.x * kTile, n0 = blockIdx.y * kTile;
   const int r16 = r < 16 ? 16 : r;                       // depth padded to the MMA's k16
   if (tid < 16) s_q[tid] = tb.q[tid];
-  s_inv127[tid] = __fdiv_rn((float)(tid - 128), 127.0f);   // entry c + 128: any int8 c
+  s_inv127[tid] = dq_code_value(tid, dq_type);             // entry c + 128: any code byte
   for (int i = tid; i < r16 * (kTile / 8); i += 256) {
     const int j = i / (kTile / 8), ch = i % (kTile / 8);
     const int k = k0 + ch * 8;
@@ -255,11 +255,11 @@ void launch_merge(const nf4_weight* w, const void* A, const void* B, int r, floa
   if (w->double_quant)
     k_qlora_merge<true><<<grid, 256, 0, st>>>(w->packed, (int)w->rows, (int)w->cols, nullptr, w->qabsmax,
                                               w->dq_scale, w->dq_mean, (const __nv_bfloat16*)A,
-                                              (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, tb);
+                                              (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, tb, w->double_quant);
   else
     k_qlora_merge<false><<<grid, 256, 0, st>>>(w->packed, (int)w->rows, (int)w->cols, w->absmax, nullptr,
                                                nullptr, nullptr, (const __nv_bfloat16*)A,
-                                               (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, tb);
+                                               (const __nv_bfloat16*)B, r, s, (__nv_bfloat16*)out, tb, 0);
 }
 
 }  // namespace qnf4

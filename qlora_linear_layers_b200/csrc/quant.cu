@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -394,6 +395,7 @@ k_dq_hist(const float* __restrict__ absmax, int64_t n, unsigned long long* __res
 // Pass 2: the mean over n_total absmax values (this array's n and any other
 // shards' absmax whose histograms were added in), then the int8 codes and
 // fp32 scales of this array's groups.
+template <int DQT>
 __global__ void __launch_bounds__(512)
 k_dq_finalize(const float* __restrict__ absmax, int64_t n, const unsigned long long* __restrict__ hist,
               int64_t n_total, int8_t* __restrict__ qabsmax, float* __restrict__ dq_scale,
@@ -442,8 +444,13 @@ k_dq_finalize(const float* __restrict__ absmax, int64_t n, const unsigned long l
       if (i < n) {
         int c = 0;
         if (m != 0.0f) {
-          c = __float2int_rn(__fmul_rn(__fdiv_rn(d[j], m), 127.0f));
-          c = min(max(c, -127), 127);
+          if (DQT == 2) {
+            // E4M3 code of 256 * RN32(d / s_g) (exact scaling), nearest, ties to even
+            c = (int)(int8_t)__nv_cvt_float_to_fp8(__fmul_rn(__fdiv_rn(d[j], m), 256.0f), __NV_SATFINITE, __NV_E4M3);
+          } else {
+            c = __float2int_rn(__fmul_rn(__fdiv_rn(d[j], m), 127.0f));
+            c = min(max(c, -127), 127);
+          }
         }
         qabsmax[i] = (int8_t)c;
       }
@@ -455,10 +462,13 @@ k_dq_finalize(const float* __restrict__ absmax, int64_t n, const unsigned long l
 // Returns the number of kernels launched.
 int launch_double_quantize_from_hist(const float* absmax, int64_t n, const unsigned long long* hist,
                                      int64_t n_total, int8_t* qabsmax, float* dq_scale, float* dq_mean,
-                                     cudaStream_t s, int num_sms) {
+                                     cudaStream_t s, int num_sms, int dq_type) {
   const int64_t ngroups = (n + 255) / 256;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((ngroups + 15) / 16, (int64_t)num_sms * 2));
-  k_dq_finalize<<<blocks, 512, 0, s>>>(absmax, n, hist, n_total, qabsmax, dq_scale, dq_mean);
+  if (dq_type == 2)
+    k_dq_finalize<2><<<blocks, 512, 0, s>>>(absmax, n, hist, n_total, qabsmax, dq_scale, dq_mean);
+  else
+    k_dq_finalize<1><<<blocks, 512, 0, s>>>(absmax, n, hist, n_total, qabsmax, dq_scale, dq_mean);
   return 1;
 }
 
@@ -468,7 +478,7 @@ int launch_double_quantize(const float* absmax, int64_t n, int8_t* qabsmax, floa
   cudaMemsetAsync(hist, 0, 256 * sizeof(unsigned long long), s);
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((n + 8191) / 8192, (int64_t)num_sms));
   k_dq_hist<<<blocks, 512, 0, s>>>(absmax, n, hist, status);
-  return 2 + launch_double_quantize_from_hist(absmax, n, hist, n, qabsmax, dq_scale, dq_mean, s, num_sms);
+  return 2 + launch_double_quantize_from_hist(absmax, n, hist, n, qabsmax, dq_scale, dq_mean, s, num_sms, 1);
 }
 
 // ===========================================================================
@@ -484,12 +494,12 @@ __global__ void __launch_bounds__(256)
 k_dequantize(const uint32_t* __restrict__ packed, int64_t nchunks,
              const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
              const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
-             uint4* __restrict__ out, CodeTables tb) {
+             uint4* __restrict__ out, CodeTables tb, int dq_type) {
   constexpr int kU = 4;
   __shared__ float s_q[16];
   __shared__ float s_inv127[256];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
-  s_inv127[threadIdx.x] = __fdiv_rn((float)((int)threadIdx.x - 128), 127.0f);   // entry c + 128: any int8 c
+  s_inv127[threadIdx.x] = dq_code_value((int)threadIdx.x, dq_type);   // entry c + 128: any code byte
   __syncthreads();
   const float mu = DQ ? dq_mean[0] : 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -527,10 +537,10 @@ void launch_dequantize(const nf4_weight* w, void* out, cudaStream_t s, int num_s
   const CodeTables& tb = host_tables(w->quant_type);
   if (w->double_quant)
     k_dequantize<true><<<blocks, 256, 0, s>>>((const uint32_t*)w->packed, nchunks, nullptr, w->qabsmax,
-                                              w->dq_scale, w->dq_mean, (uint4*)out, tb);
+                                              w->dq_scale, w->dq_mean, (uint4*)out, tb, w->double_quant);
   else
     k_dequantize<false><<<blocks, 256, 0, s>>>((const uint32_t*)w->packed, nchunks, w->absmax, nullptr,
-                                               nullptr, nullptr, (uint4*)out, tb);
+                                               nullptr, nullptr, (uint4*)out, tb, 0);
 }
 
 }  // namespace qnf4

@@ -729,3 +729,44 @@ def test_dropout_layer_vs_autograd():
     np.testing.assert_allclose(dX, Xt.grad.numpy(), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(dA, At.grad.numpy(), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(dB, Bt.grad.numpy(), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit float double quantisation
+# ---------------------------------------------------------------------------
+
+def test_e4m3_encode_matches_torch():
+    """The oracle's E4M3 rounding equals torch's float8_e4m3fn cast (round to
+    nearest, ties to even) on random values, every representable value and
+    every midpoint between neighbours (|x| <= 448, where the cast does not
+    saturate)."""
+    v = oracle.e4m3_values()
+    mids = (v[:-1] + v[1:]) / 2
+    rng = np.random.default_rng(12)
+    x = np.concatenate([v, mids, -v, -mids, rng.uniform(-300, 300, 5000),
+                        rng.standard_normal(5000) * 1e-2]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_encode(x)
+    assert np.array_equal(got, want)
+    assert np.array_equal(oracle.e4m3_decode(got), torch.from_numpy(got).view(torch.float8_e4m3fn).double().numpy())
+    assert oracle.e4m3_values()[-1] == 448.0 and oracle.e4m3_values().size == 127
+
+
+def test_double_quantize_fp8_properties():
+    """fp8 variant: the group max maps to code 256 (0x78 = 2^8, t = +/-1
+    exactly), and the recovered scales are within E4M3's half-ulp relative
+    error of d plus rounding."""
+    rng = np.random.default_rng(16)
+    a = (np.abs(rng.standard_normal(1000)) * 0.05).astype(np.float32)
+    q, s, mu = oracle.double_quantize(a, fmt="fp8")
+    d = (a - mu).astype(np.float32)
+    for g in range(4):
+        dg = d[g * 256:(g + 1) * 256]
+        i = int(np.argmax(np.abs(dg)))
+        assert (q[g * 256 + i].view(np.uint8) & 0x7F) == 0x78
+    ah = oracle.dq_absmax(q, s, mu, fmt="fp8")
+    sg = np.repeat(s, 256)[:a.size].astype(np.float64)
+    bound = np.abs(d).astype(np.float64) * 2.0 ** -4 + sg * 2.0 ** -17 + 4 * np.spacing(np.abs(a))
+    assert np.all(np.abs(ah.astype(np.float64) - a) <= bound)
+    q8, _, _ = oracle.double_quantize(a)
+    assert not np.array_equal(q, q8)

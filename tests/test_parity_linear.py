@@ -39,8 +39,9 @@ def _oracle_weight(wq, W_cpu):
     table = oracle.fp4_table() if wq.quant_type == 1 else oracle.nf4_table()
     codes, a = oracle.quantize(W_cpu.float().numpy(), table)
     if wq.double_quant:
-        qa, s, mu = oracle.double_quantize(a)
-        a = oracle.dq_absmax(qa, s, mu)
+        fmt = "fp8" if int(wq.double_quant) == 2 else "int8"
+        qa, s, mu = oracle.double_quantize(a, fmt=fmt)
+        a = oracle.dq_absmax(qa, s, mu, fmt=fmt)
     return oracle.dequantize(oracle.pack(codes), a, tuple(W_cpu.shape), table=table)
 
 
@@ -118,12 +119,34 @@ def test_forward_small_fp4(q, N, K, M, r, alpha, dq):
     assert rel_err(T, Tr) <= TOL
 
 
-@pytest.mark.parametrize("qt", [0, 1])
-def test_forward_identity_is_exact_dequant(q, qt):
+@pytest.mark.parametrize("N,K,M,r,alpha", [
+    (384, 512, 300, 16, 32.0),
+    (96, 256, 300, 16, 32.0),
+    (512, 1024, 4, 16, 32.0),
+])
+def test_forward_backward_fp8_scales(q, N, K, M, r, alpha):
+    """Block scales double-quantised to E4M3 codes (double_quant = 2) in the
+    forward GEMM engines, the decode kernel and the backward."""
+    W, X, A, B, wq = _layer(q, N, K, M, r, alpha, seed=500 + M + r, dq=2)
+    dY = synth.activations(M, N, 511 + M)
+    Xc, Ac, Bc, dYc = X.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    Y, T = q.linear_fwd(wq, Xc, Ac, Bc, alpha)
+    dX, dA, dB = q.linear_bwd(wq, Xc, dYc, Ac, Bc, alpha, T=T)
+    assert q.qlora_check_status() == 0
+    Wd = _oracle_weight(wq, W)
+    Xn, An, Bn, dYn = (t.float().numpy() for t in (X, A, B, dY))
+    Yr, Tr = oracle.linear_fwd(Xn, Wd, An, Bn, alpha, r)
+    dXr, dAr, dBr = oracle.linear_bwd(Xn, dYn, Wd, An, Bn, alpha, r)
+    assert rel_err(Y, Yr) <= TOL and rel_err(T, Tr) <= TOL
+    assert rel_err(dX, dXr) <= TOL and rel_err(dA, dAr) <= TOL and rel_err(dB, dBr) <= TOL
+
+
+@pytest.mark.parametrize("qt,dq", [(0, 1), (1, 1), (0, 2)])
+def test_forward_identity_is_exact_dequant(q, qt, dq):
     """X = I, A = 0: Y[m, n] = W'[n, m] exactly (one nonzero product per sum)."""
     N, K = 384, 512
     W = synth.weight(N, K, 4242, "bf16")
-    wq = q.quantize(W.cuda(), double_quant=True, quant_type=qt)
+    wq = q.quantize(W.cuda(), double_quant=dq, quant_type=qt)
     X = torch.eye(K, dtype=torch.bfloat16, device="cuda")
     A = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
     B = synth.activations(N, 16, 4243, sigma=0.02).cuda()

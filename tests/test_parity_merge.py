@@ -31,8 +31,9 @@ def _oracle_deq(W_cpu, dq, qt):
     table = oracle.fp4_table() if qt == 1 else oracle.nf4_table()
     codes, a = oracle.quantize(W_cpu.float().numpy(), table)
     if dq:
-        qa, s, mu = oracle.double_quantize(a)
-        a = oracle.dq_absmax(qa, s, mu)
+        fmt = "fp8" if int(dq) == 2 else "int8"
+        qa, s, mu = oracle.double_quantize(a, fmt=fmt)
+        a = oracle.dq_absmax(qa, s, mu, fmt=fmt)
     return oracle.dequantize(oracle.pack(codes), a, tuple(W_cpu.shape), table=table)
 
 
@@ -50,6 +51,7 @@ def _check(got, ref):
     (136, 320, 128, 64.0, False, 0),
     (1024, 1024, 16, 32.0, True, 0),
     (256, 640, 32, 8.0, True, 1),          # FP4 storage
+    (384, 512, 64, 16.0, 2, 0),            # E4M3 block-scale codes
 ])
 def test_merge_small(q, N, K, r, alpha, dq, qt):
     W = synth.weight(N, K, 600 + r, "bf16")

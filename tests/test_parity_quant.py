@@ -49,11 +49,12 @@ def _check_full(q, W_cpu, double_quant=True, qt=NF4):
     assert np.array_equal(_np(wq.packed), oracle.pack(codes))
     assert np.array_equal(_np(wq.absmax).view(np.uint32), a.view(np.uint32))
     if double_quant:
-        qa, s, mu = oracle.double_quantize(a)
+        fmt = "fp8" if int(double_quant) == 2 else "int8"
+        qa, s, mu = oracle.double_quantize(a, fmt=fmt)
         assert np.array_equal(_np(wq.qabsmax), qa)
         assert np.array_equal(_np(wq.dq_scale).view(np.uint32), s.view(np.uint32))
         assert _np(wq.dq_mean)[0].view(np.uint32) == np.float32(mu).view(np.uint32)
-        ah = oracle.dq_absmax(qa, s, mu)
+        ah = oracle.dq_absmax(qa, s, mu, fmt=fmt)
     else:
         ah = a
     ref = oracle.dequantize(oracle.pack(codes), ah, Wnp.shape, table=table)
@@ -75,6 +76,16 @@ def test_attn_proj_bf16(q, qt):
     wl = synth.WORKLOADS["attn_proj_4096"]
     W = synth.weight(4096, 4096, wl.seed(synth.TID_W), "bf16")
     _check_full(q, W, True, qt)
+
+
+@pytest.mark.parametrize("rows,cols,outliers", [(4096, 4096, False), (300, 4096, True), (5, 64 * 257, False)])
+def test_fp8_double_quant(q, rows, cols, outliers):
+    """8-bit float block-scale codes (double_quant = 2): codes, E4M3 scale
+    bytes (signed zeros included), group scales, mean and the dequantised
+    weights bit for bit."""
+    W = synth.weight(rows, cols, 880 + rows, "bf16", outliers=outliers)
+    _check_full(q, W, 2)
+    _check_full(q, W, 2, FP4)
 
 
 @pytest.mark.parametrize("rows,cols", [(1, 64), (3, 6400), (7, 192), (5, 64 * 257)])
