@@ -461,59 +461,62 @@ size_t atb_workspace_floats(int Rdim, int Cdim, int M) {
 // row; 256 threads, each dequantises 32 weights into shared memory, then the
 // tile is written out transposed with 16-byte stores.
 // ===========================================================================
+// Dequantise-transpose: Wt[k, n] = deq(W)[n, k], bf16, same values as
+// nf4_dequantize.  CTA tile 64 rows (n) x 128 columns (k) = 2 NF4 blocks per
+// row; thread (p, q) expands rows 2p and 2p + 1, columns [16q, 16q + 16), and
+// stores each column's pair of rows as one 32-bit word of the transposed tile
+// in shared memory (a warp's 32 words are consecutive: no bank conflicts);
+// the CTA then writes the tile's 128 rows of 128 bytes with 16-byte stores.
+// ===========================================================================
 __global__ void __launch_bounds__(256)
 k_dequant_t(const uint8_t* __restrict__ packed, int N, int K, int dq,
             const float* __restrict__ absmax, const int8_t* __restrict__ qabsmax,
             const float* __restrict__ dq_scale, const float* __restrict__ dq_mean,
             __nv_bfloat16* __restrict__ Wt, CodeTables tb) {
-  __shared__ uint16_t tile[64][128 + 8];
+  constexpr int kPitch = 36;                       // words per transposed row (32 + pad, 16-byte rows)
+  __shared__ __align__(16) uint32_t tileT[128 * kPitch];
   __shared__ float s_q[16];
   if (threadIdx.x < 16) s_q[threadIdx.x] = tb.q[threadIdx.x];
-  __syncthreads();
   const int n0 = blockIdx.y * 64, k0 = blockIdx.x * 128;
   const int tid = threadIdx.x;
-  {
-    const int row = tid >> 2, part = tid & 3;        // 4 threads x 32 weights per row
-    const int n = n0 + row, k = k0 + part * 32;
-    if (n < N && k < K) {
-      const int64_t e = (int64_t)n * K + k;
-      const int64_t blk = e >> 6;
-      float a;
-      if (dq) {
-        a = __fadd_rn(__fmul_rn(dq_code_value((int)qabsmax[blk] + 128, dq), dq_scale[blk >> 8]), dq_mean[0]);
-      } else {
-        a = absmax[blk];
-      }
-      const uint4 pk = *reinterpret_cast<const uint4*>(packed + (e >> 1));
-      const uint32_t wds[4] = {pk.x, pk.y, pk.z, pk.w};
+  const int pr = tid & 31, qk = tid >> 5;          // row pair, 16-column group
+  // codes and scales of rows 2pr, 2pr + 1 (clamped: rows past N write zeros)
+  uint2 cw[2];
+  float a[2];
+  const int k = k0 + 16 * qk;
+  const bool kin = k < K;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const uint32_t byte = (wds[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-        const uint32_t v = pack_bf16x2(__fmul_rn(s_q[byte >> 4], a), __fmul_rn(s_q[byte & 15], a));
-        tile[row][part * 32 + 2 * j] = (uint16_t)(v & 0xFFFF);
-        tile[row][part * 32 + 2 * j + 1] = (uint16_t)(v >> 16);
-      }
-    } else {
+  for (int h = 0; h < 2; ++h) {
+    const int n = n0 + 2 * pr + h;
+    const bool in = kin && n < N;
+    const int64_t e = (int64_t)(in ? n : 0) * K + (in ? k : 0);
+    cw[h] = in ? *reinterpret_cast<const uint2*>(packed + (e >> 1)) : make_uint2(0u, 0u);
+    const int64_t blk = e >> 6;
+    if (!in) a[h] = 0.0f;
+    else if (dq) a[h] = __fadd_rn(__fmul_rn(dq_code_value((int)qabsmax[blk] + 128, dq), dq_scale[blk >> 8]), dq_mean[0]);
+    else a[h] = absmax[blk];
+  }
+  __syncthreads();                                 // s_q
 #pragma unroll
-      for (int j = 0; j < 32; ++j) tile[row][part * 32 + j] = 0;
-    }
+  for (int b = 0; b < 8; ++b) {                    // code byte b: columns 2b (high nibble), 2b + 1
+    const uint32_t c0 = ((b < 4 ? cw[0].x : cw[0].y) >> (8 * (b & 3))) & 0xFFu;
+    const uint32_t c1 = ((b < 4 ? cw[1].x : cw[1].y) >> (8 * (b & 3))) & 0xFFu;
+    const uint32_t even = pack_bf16x2(__fmul_rn(s_q[c0 >> 4], a[0]), __fmul_rn(s_q[c1 >> 4], a[1]));
+    const uint32_t odd = pack_bf16x2(__fmul_rn(s_q[c0 & 15], a[0]), __fmul_rn(s_q[c1 & 15], a[1]));
+    tileT[(16 * qk + 2 * b) * kPitch + pr] = even;
+    tileT[(16 * qk + 2 * b + 1) * kPitch + pr] = odd;
   }
   __syncthreads();
-  {
-    // 128 output rows (k) x 64 columns (n): 2 threads per row, 32 n each
-    const int kr = tid >> 1, half = tid & 1;
-    const int k = k0 + kr;
-    if (k < K) {
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int nb = half * 32 + v * 8;
-        if (n0 + nb >= N) break;
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          w[j] = (uint32_t)tile[nb + 2 * j][kr] | ((uint32_t)tile[nb + 2 * j + 1][kr] << 16);
-        *reinterpret_cast<uint4*>(Wt + (int64_t)k * N + n0 + nb) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+  const bool full_n = n0 + 64 <= N;
+  for (int i = tid; i < 128 * 8; i += 256) {
+    const int kr = i >> 3, ch = i & 7;             // transposed row, 16-byte chunk (8 columns n)
+    const int kk = k0 + kr, nn = n0 + ch * 8;
+    if (kk >= K) continue;
+    const uint4 v = *reinterpret_cast<const uint4*>(&tileT[kr * kPitch + ch * 4]);
+    if (full_n || nn + 8 <= N) {
+      *reinterpret_cast<uint4*>(Wt + (int64_t)kk * N + nn) = v;
+    } else if (nn < N) {                           // N % 8 == 0: never partial
+      *reinterpret_cast<uint4*>(Wt + (int64_t)kk * N + nn) = v;
     }
   }
 }
