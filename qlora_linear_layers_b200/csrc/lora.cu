@@ -210,13 +210,14 @@ __global__ void k_skinny_reduce(const float* __restrict__ part, int splits, int 
   }
 }
 
-// Number of contraction slices for an M x L skinny product: enough CTAs to
-// cover the GPU twice over (~296), whatever the device, so that the workspace
-// size and summation order depend only on the shapes.
+// Number of contraction slices for an M x L skinny product: about one full
+// wave of CTAs on a B200 (148 SMs x 3 resident CTAs), whatever the device, so
+// that the workspace size and summation order depend only on the shapes.
+constexpr int kOneWave = 148 * 3;
 int skinny_splits(int M, int L) {
   const int tiles = (M + 127) / 128;
   const int nkc = (L + 63) / 64;
-  int splits = std::min(std::max(1, (296 + tiles - 1) / tiles), nkc);
+  int splits = std::min(std::max(1, kOneWave / tiles), nkc);
   const int cps = (nkc + splits - 1) / splits;
   return (nkc + cps - 1) / cps;
 }
@@ -406,10 +407,11 @@ __global__ void k_reduce_partials(const float* __restrict__ part, int nchunks, i
   }
 }
 
-// Split count of the token dimension: aims at ~600 CTAs whatever the device,
-// so that workspace size and summation order depend only on the shapes.
+// Split count of the token dimension: about one full wave of CTAs on a B200
+// (148 SMs x 3 resident CTAs) whatever the device, so that workspace size and
+// summation order depend only on the shapes.
 int atb_chunks(int tiles, int M) {
-  int want = std::max(1, (600 + tiles - 1) / tiles);
+  int want = std::max(1, kOneWave / tiles);
   int maxc = std::max(1, (M + 31) / 32);
   return std::min(want, maxc);
 }
