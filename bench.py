@@ -46,13 +46,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA NF4 linear TFLOP/s & quant/dequant GB/s, % of B200 roofline"
-# DRAM bytes (read + write) per launch of the fused forward GEMM on this
-# workload, averaged over the step's three launches, from one ncu capture of
-# each shape (dram__bytes_read.sum + dram__bytes_write.sum of
-# `bench.py --case fwd --tokens 8192 --proj 0|2`).  None until the current
-# kernel has been captured: the figure is reported only for the kernel it
-# was measured on.  The algorithmic bytes are 407 MB per launch.
-FWD_GEMM_DRAM_BYTES_PER_LAUNCH = None
+# DRAM bytes (read + write) per launch of the fused forward GEMM
+# (k_qlora_gemm_dual) on this workload, averaged over the step's three
+# launches, from one ncu capture of each shape (dram__bytes_read.sum +
+# dram__bytes_write.sum of `bench.py --case fwd --tokens 8192 --proj 0|2`):
+# gate and up 369.9 MB, down 537.4 MB.  Set back to None when the
+# kernel changes: the figure belongs to the kernel it was measured on.  The
+# algorithmic bytes are about 405 MB per launch.
+FWD_GEMM_DRAM_BYTES_PER_LAUNCH = (369.9e6 * 2 + 537.4e6) / 3
 WORKLOAD = "mlp_7b"
 DECODE_M = 16
 
