@@ -374,7 +374,7 @@ def run_ours(args, rank, world, local_rank):
     # peak is the denominator; the sustained peak is reported beside it.
     gemm_flops = [2 * M * N * K + 2 * M * N * r for (N, K) in wl.weights]
     achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
-    roofline = {"kernel": "k_qlora_gemm_pair<NF4> (fused NF4-dequant forward GEMM + adapter tail, paired SMs)",
+    roofline = {"kernel": "k_qlora_gemm_dual (fused NF4-dequant forward GEMM, two token tiles per weight stage, adapter as extra K steps, paired SMs)",
                 "bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
                 "frac": achieved / tc_burst, "traffic": FWD_GEMM_DRAM_BYTES_PER_LAUNCH,
                 "peak_kind": f"bf16 dense, burst ({pk['source']}); the timed region lasts "
