@@ -222,9 +222,10 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
       // consumers' bounded waits run out (QLORA_ERR_TIMEOUT)
       const bool withhold = blockIdx.x == 0 &&
                             reinterpret_cast<const volatile DevState*>(p.status)->withhold_first_fill != 0;
-      for (int64_t u = u0; u < u1; ++u, ++k) {
-        const int s = (int)(k % kStages);
-        if (!(ok = mbar_wait(&S.empty[s], ((k / kStages) & 1) ^ 1, abort, p.status))) break;
+      int s = 0;
+      uint32_t ph = 0;                           // phase of stage s's current use
+      for (int64_t u = u0; u < u1; ++u, ++k, s = (s + 1 == kStages) ? 0 : s + 1, ph ^= (s == 0)) {
+        if (!(ok = mbar_wait(&S.empty[s], ph ^ 1, abort, p.status))) break;
         const int b = st * kBlk;
         uint8_t* dst = stage_ptr(s);
         if (withhold && k == 0) {
@@ -342,7 +343,9 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     if (u0 + d < u1) load_scales(prgp, pst, sq[d], sf[d]);
     if (++pst == p.spr) { pst = 0; ++prgp; }
   }
-  for (int64_t u = u0; u < u1; ++u, ++k) {
+  int s = 0;
+  uint32_t ph = 0;                               // phase of stage s's current use
+  for (int64_t u = u0; u < u1; ++u, ++k, s = (s + 1 == kStages) ? 0 : s + 1, ph ^= (s == 0)) {
     const int b = st * kBlk + j;
     int nrgp = rgp, nst = st + 1;                 // the next unit
     if (nst == p.spr) { nst = 0; ++nrgp; }
@@ -356,8 +359,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     for (int d = 0; d + 1 < kAhead; ++d) { sq[d] = sq[d + 1]; sf[d] = sf[d + 1]; }
     if (u + kAhead < u1) load_scales(prgp, pst, sq[kAhead - 1], sf[kAhead - 1]);
     if (++pst == p.spr) { pst = 0; ++prgp; }
-    const int s = (int)(k % kStages);
-    if (!(ok = mbar_wait(&S.full[s], (k / kStages) & 1, abort, p.status))) break;
+    if (!(ok = mbar_wait(&S.full[s], ph, abort, p.status))) break;
     const uint8_t* sb = stage_ptr(s);
     const bool nf4 = rgp >= p.nat;
     if (b < p.nb && (nf4 || h == 0)) {

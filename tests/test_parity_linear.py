@@ -158,6 +158,36 @@ def test_forward_identity_is_exact_dequant(q, qt, dq):
     assert np.array_equal(Y.t().float().cpu().numpy(), Wd)
 
 
+@pytest.mark.parametrize("qt,dq,M", [(0, 1, 1), (0, 1, 16), (1, 1, 9), (0, 2, 4), (0, 0, 8)])
+def test_decode_onehot_tokens_exact(q, qt, dq, M):
+    """Decode path (M <= 16) with one-hot token rows and A = 0: every output
+    is one table value times one block scale, so Y equals, bit for bit, the
+    decode path's reading of the weight, RNbf16(RN32(a^ * RNbf16(q[c]))) --
+    which pins its row, block and column mapping and its scale decode."""
+    N, K = 384, 1024
+    W = synth.weight(N, K, 4300 + M, "bf16")
+    wq = q.quantize(W.cuda(), double_quant=dq, quant_type=qt)
+    cols = np.random.default_rng(M).choice(K, M, replace=False)
+    X = torch.zeros(M, K, dtype=torch.bfloat16)
+    X[np.arange(M), torch.from_numpy(cols)] = 1.0
+    A = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
+    B = synth.activations(N, 16, 4301, sigma=0.02).cuda()
+    Y, _ = q.linear_fwd(wq, X.cuda(), A, B, 32.0)
+    assert q.qlora_check_status() == 0
+    table = oracle.fp4_table() if qt == 1 else oracle.nf4_table()
+    codes, a = oracle.quantize(W.float().numpy(), table)
+    if dq:
+        fmt = "fp8" if dq == 2 else "int8"
+        a = oracle.dq_absmax(*oracle.double_quantize(a, fmt=fmt), fmt=fmt)
+    codes = np.asarray(codes).reshape(N, K)
+    ah = np.asarray(a, dtype=np.float32).reshape(N, K // 64)
+    qb = oracle.round_bf16(np.asarray(table, dtype=np.float32))
+    Yg = Y.float().cpu().numpy()
+    for m, k in enumerate(cols):
+        expect = oracle.round_bf16((ah[:, k // 64] * qb[codes[:, k]]).astype(np.float32))
+        assert np.array_equal(Yg[m], expect), (m, k)
+
+
 def test_forward_adapter_only(q):
     """W = 0 quantises to the exact-zero row everywhere: Y = s (X A^T) B^T."""
     N, K, M, r, alpha = 256, 512, 300, 16, 32.0
