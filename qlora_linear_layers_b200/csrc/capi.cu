@@ -519,7 +519,7 @@ static int bwd_impl(const nf4_weight* w, const void* X, const void* dY, int64_t 
   cudaEvent_t e0, e1;
   take_gemm_events(&e0, &e1);
   if (e0) cudaEventRecord(e0, s);
-  st = K > 128 ? launch_qlora_gemm_pair(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms)
+  st = K > 128 ? launch_qlora_gemm_pair(a, dY, sU, At, Wt, RP, s, d->sms)
                : launch_qlora_gemm(MODE_BF16, a, dY, sU, At, Wt, RP, s, d->sms);
   if (e1) cudaEventRecord(e1, s);
   if (st) return st;

@@ -31,11 +31,11 @@ struct GemmArgs {
   float q[16];                // NF4 table
 };
 
-// Paired-SM (cluster of 2, tcgen05 cta_group::2) form of the GEMM: 256 x 256
-// output tiles; tok: [Mtok, Kc]; tokad: [Mtok, RP]; MODE_NF4 weights from
-// `a`, MODE_BF16 weights w [Nout, Kc] and wad [Nout, RP].
-int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
-                           const void* wad, const void* w, int RP, cudaStream_t s, int num_sms);
+// Backward dX GEMM on SM pairs (cluster of 2, tcgen05 cta_group::2): 256 x BM
+// output tiles; tok: [Mtok, Kc]; tokad: [Mtok, RP]; weights w [Nout, Kc] and
+// wad [Nout, RP] bf16.
+int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad, const void* wad,
+                           const void* w, int RP, cudaStream_t s, int num_sms);
 
 // Forward NF4 GEMM on SM pairs with two token tiles per weight tile (the
 // weights of a stage are dequantised once into shared memory and feed two

@@ -1,27 +1,23 @@
-// QLoRA GEMMs on paired SMs (tcgen05 cta_group::2).
+// Backward dX GEMM on paired SMs (tcgen05 cta_group::2):
 //
-//   MODE_NF4  (forward):      Y  = X deq(W)^T + (s T) B^T
-//   MODE_BF16 (backward dX):  dX = dY deq(W) + (s U) A     (weights as deq(W)^T, bf16)
+//   dX = dY deq(W) + (s U) A     (weights supplied as deq(W)^T, bf16)
 //
-// Same computation and layout rules as the single-CTA engine in gemm.cu (page
-// "QLoRA Explained", section "Why the expansion cannot be skipped": codes ->
-// table -> block scale -> bf16 -> tensor core), with two SMs of a cluster
-// sharing each 256 x 256 output tile:
-//  * MMA M = 256 (CTA r owns weight rows 128r..128r+127 of the tile, written
-//    by its own converter warps into its own TMEM), MMA N = 256 (CTA r loads
-//    tokens 128r..128r+127 of the tile into its own shared memory).  Each SM
-//    thus streams half the token tile per K step that a single-CTA 128 x 256
-//    tile needs, halving the shared-memory port traffic (TMA writes + MMA
-//    reads of the token operand), which is what bounds the single-CTA kernel.
-//  * The even CTA's elected thread issues tcgen05.mma.cta_group::2 and
-//    commits with an arrival multicast to both CTAs' "empty" and "full"
-//    barriers.  Both CTAs' TMA loads (no multicast: each CTA loads its own
-//    half) complete on the even CTA's "full" barrier; the odd CTA's converter
-//    and epilogue warps arrive on the even CTA's barriers through mapa.
-//  * MODE_NF4: 8 pipeline stages of 16 KB of tokens per CTA, A ring of 8 x 32
-//    TMEM columns beside the 256-column accumulator (all 512 columns).
-//  * MODE_BF16: both operands by TMA (each CTA its 128 weight rows and its
-//    128 tokens), 6 stages of 16 + 16 KB; the converter warps stay idle.
+// Page "QLoRA Explained", config walk-through: the input gradient flows
+// through the frozen 4-bit base (dequantised, never updated) and the adapter.
+// Two SMs of a cluster share each 256 x BM output tile:
+//  * MMA M = 256 (CTA r owns weight rows 128r..128r+127 of the tile), MMA N =
+//    BM (CTA r loads tokens BM/2 r..BM/2 r + BM/2 - 1).  Each SM streams half
+//    the token tile per K step, halving the shared-memory port traffic (TMA
+//    writes + MMA reads of the token operand).
+//  * Both operands arrive by TMA (each CTA its 128 weight rows and its BM/2
+//    tokens), 6 stages of 16 + 16 KB; the adapter term runs as RP/64 extra K
+//    steps over [s U | A^T].
+//  * The even CTA's elected thread issues tcgen05.mma.cta_group::2 with both
+//    operands in shared memory and commits with an arrival multicast to both
+//    CTAs' "empty" and "full" barriers.  Both CTAs' TMA loads (no multicast:
+//    each CTA loads its own half) complete on the even CTA's "full" barrier;
+//    the odd CTA's epilogue warps arrive on the even CTA's barriers through
+//    mapa.
 // Every wait is bounded (status QLORA_ERR_TIMEOUT); both CTAs meet at a
 // cluster barrier before the paired TMEM is released.
 
@@ -33,56 +29,49 @@
 
 #include "common.cuh"
 #include "gemm.h"
-#include "nf4_lut.cuh"
 
 namespace qnf4 {
 
 namespace pair {
 
 constexpr int BN = 128;          // weight rows per CTA (MMA M = 256 per pair)
-constexpr int BK = 64;           // contraction per stage (= one NF4 block)
-template <int MODE> __host__ __device__ constexpr int stages() { return MODE == MODE_NF4 ? 8 : 6; }
+constexpr int BK = 64;           // contraction per stage
+constexpr int NS = 6;            // pipeline stages
 // BM (template argument, a multiple of 32 up to 256): tokens per pair tile =
 // MMA N; each CTA loads BM / 2 tokens, BM * 64 bytes per stage.
 constexpr int ACC_COL = 0;                       // accumulator: TMEM columns [0, 256)
-constexpr int A_COL = 256;                       // MODE_NF4 A ring: 8 x 32 columns
-constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 448;                 // 14 warps
-constexpr int CVT_WARP0 = 6;                     // warps 6-13: A-operand producers
+constexpr int TMEM_COLS = 256;
+constexpr int NUM_THREADS = 192;                 // warp 0 TMA, 1 MMA, 2-5 epilogue
 constexpr uint16_t kBoth = 0x3;                  // cluster CTA mask of the pair
 
-constexpr int W_BYTES = BN * BK * 2;             // 16 KB weight tile per CTA (MODE_BF16)
+constexpr int W_BYTES = BN * BK * 2;             // 16 KB weight tile per CTA and stage
 
-template <int MODE, int BM>
+template <int BM>
 struct Smem {
-  static constexpr int NS = stages<MODE>();
   uint8_t x[NS][BM * BK];
-  uint8_t w[MODE == MODE_BF16 ? NS : 1][MODE == MODE_BF16 ? W_BYTES : 16];
+  uint8_t w[NS][W_BYTES];
   uint64_t x_full[NS], x_empty[NS];
-  uint64_t a_full[NS], a_empty[NS];
   uint64_t acc_full, acc_empty, done;
   uint32_t tmem_base;
   int abort;
-  float inv127[256];
 };
 
-template <int MODE, int BM>
-constexpr size_t smem_bytes() { return sizeof(Smem<MODE, BM>) + 1024; }
+template <int BM>
+constexpr size_t smem_bytes() { return sizeof(Smem<BM>) + 1024; }
 
-template <int MODE, bool DQ, int BM>
+template <int BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc]  bf16
                   const __grid_constant__ CUtensorMap tm_tokad,   // [Mtok, RP]  bf16
-                  const __grid_constant__ CUtensorMap tm_w,       // [Nout, Kc]  bf16 (MODE_BF16)
-                  const __grid_constant__ CUtensorMap tm_wad,     // [Nout, RP]  bf16 (MODE_BF16)
+                  const __grid_constant__ CUtensorMap tm_w,       // [Nout, Kc]  bf16
+                  const __grid_constant__ CUtensorMap tm_wad,     // [Nout, RP]  bf16
                   const GemmArgs p) {
   static_assert(BM % 32 == 0 && BM >= 32 && BM <= 256, "token tile");
-  constexpr int NS = stages<MODE>();
   constexpr int BMH = BM / 2;                      // tokens loaded by each CTA
   constexpr int X_BYTES = BMH * BK * 2;
   extern __shared__ uint8_t smem_raw[];
-  Smem<MODE, BM>& S =
-      *reinterpret_cast<Smem<MODE, BM>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<BM>& S =
+      *reinterpret_cast<Smem<BM>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();        // 0: issues the MMAs
@@ -99,8 +88,6 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     for (int i = 0; i < NS; ++i) {
       mbar_init(&S.x_full[i], 1);                  // leader's expect_tx; tx from both CTAs
       mbar_init(&S.x_empty[i], 1);                 // multicast commit
-      mbar_init(&S.a_full[i], 8);                  // 4 converter warps per CTA
-      mbar_init(&S.a_empty[i], 1);                 // multicast commit
     }
     mbar_init(&S.acc_full, 1);                     // multicast commit
     mbar_init(&S.acc_empty, 8);                    // 4 epilogue warps per CTA
@@ -108,8 +95,6 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
     S.abort = 0;
     mbar_fence_init();
   }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    S.inv127[i] = dq_code_value(i, p.double_quant);     // entry c + 128: any code byte
   if (warp == 1) {
     tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
     tmem_relinquish_pair();
@@ -117,10 +102,8 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_tok);
     tma_prefetch_desc(&tm_tokad);
-    if (MODE == MODE_BF16) {
-      tma_prefetch_desc(&tm_w);
-      tma_prefetch_desc(&tm_wad);
-    }
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_wad);
   }
   tc_fence_before();
   cluster_sync();                                  // barriers of both CTAs initialised
@@ -139,12 +122,12 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
         for (int ks = 0; ks < nsteps; ++ks, ++xi) {
           const int s = xi % NS;
           if (!(ok = mbar_wait_cluster(&S.x_empty[s], ((xi / NS) & 1) ^ 1, abort, p.status))) break;
-          if (leader) mbar_arrive_expect_tx(&S.x_full[s], 2 * (X_BYTES + (MODE == MODE_BF16 ? W_BYTES : 0)));
+          if (leader) mbar_arrive_expect_tx(&S.x_full[s], 2 * (X_BYTES + W_BYTES));
           const bool ad = ks >= nk;
           const int kc = (ad ? ks - nk : ks) * BK;
           const uint32_t full0 = mapa_shared(smem_u32(&S.x_full[s]), 0);
           tma_load_2d_pair(S.x[s], ad ? &tm_tokad : &tm_tok, full0, kc, m0);
-          if (MODE == MODE_BF16) tma_load_2d_pair(S.w[s], ad ? &tm_wad : &tm_w, full0, kc, n0);
+          tma_load_2d_pair(S.w[s], ad ? &tm_wad : &tm_w, full0, kc, n0);
         }
       }
     }
@@ -162,107 +145,21 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
           const int s = xi % NS;
           const uint32_t par = (xi / NS) & 1;
           ok = mbar_wait_cluster(&S.x_full[s], par, abort, p.status);
-          if (ok && MODE == MODE_NF4) ok = mbar_wait_cluster(&S.a_full[s], par, abort, p.status);
           if (!ok) break;
           tc_fence_after();
           const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.x[s]));
-          if (MODE == MODE_NF4) {
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[s]));
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              mma_ts_pair(tmem + ACC_COL, tmem + A_COL + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2),
-                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-            mma_commit_pair_mc(&S.x_empty[s], kBoth);
-            mma_commit_pair_mc(&S.a_empty[s], kBoth);
-          } else {
-            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.w[s]));
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              mma_ss_pair(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
-                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-            mma_commit_pair_mc(&S.x_empty[s], kBoth);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ss_pair(tmem + ACC_COL, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+                        idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_pair_mc(&S.x_empty[s], kBoth);
         }
         if (ok) mma_commit_pair_mc(&S.acc_full, kBoth);
       }
       // all MMAs issued by this thread are complete once `done` flips
       mma_commit_pair_mc(&S.done, 0x1);
       mbar_wait(&S.done, 0, abort, p.status);
-    }
-  } else if (warp >= CVT_WARP0) {
-    // ------------------------------------------------------------ A-operand producers (TMEM)
-    // MODE_NF4 only.  Step ks < nk: NF4 -> bf16 for block ks of the thread's
-    // weight row; step ks >= nk: 64 bf16 of the row's adapter factor B
-    // (zero-padded to RP).
-    if (MODE == MODE_NF4) {
-    const int quad = warp & 3;
-    const uint32_t par = (uint32_t)((warp - CVT_WARP0) >> 2);   // steps of this parity
-    const int row_in_tile = quad * 32 + lane;
-    const uint32_t tmem_lane = (uint32_t)(quad * 32) << 16;
-    const float mu = DQ ? __ldg(p.dq_mean) : 0.0f;
-    const int64_t kb_per_row = p.Kc / 64;
-    struct Src { uint4 c[8]; float a_raw, sg; int qa; bool valid, ad; };
-    auto fetch = [&](uint32_t ai, Src& d) -> bool {
-      const uint32_t lt = ai / (uint32_t)nsteps;
-      const int ks = (int)(ai - lt * (uint32_t)nsteps);
-      const int tile = cluster + (int)lt * n_clusters;
-      if (tile >= n_tiles) return false;
-      const int n = (tile % n_pairs_n) * (2 * BN) + (int)rank * BN + row_in_tile;
-      d.valid = n < p.Nout;
-      d.ad = ks >= nk;
-      const int64_t nn = d.valid ? n : 0;
-      if (d.ad) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.wad + nn * p.RP + (ks - nk) * BK);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) d.c[i] = __ldcg(src + i);
-      } else {
-        const uint4* codes = reinterpret_cast<const uint4*>(p.packed + nn * (p.Kc / 2)) + 2 * ks;
-        d.c[0] = __ldcg(codes);
-        d.c[1] = __ldcg(codes + 1);
-        const int64_t b = nn * kb_per_row + ks;
-        if (DQ) { d.qa = __ldcg(p.qabsmax + b); d.sg = __ldg(p.dq_scale + (b >> 8)); d.a_raw = 0.f; }
-        else { d.a_raw = __ldcg(p.absmax + b); d.qa = 0; d.sg = 0.f; }
-      }
-      return true;
-    };
-    Src cur, nxt;
-    uint32_t ai = par;
-    bool have = fetch(ai, cur);
-    while (have) {
-      const bool more = fetch(ai + 2, nxt);       // prefetch this warp's next step
-      uint32_t v[32];
-      if (!cur.valid) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0u;
-      } else if (cur.ad) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[4 * i] = cur.c[i].x; v[4 * i + 1] = cur.c[i].y;
-          v[4 * i + 2] = cur.c[i].z; v[4 * i + 3] = cur.c[i].w;
-        }
-      } else {
-        // a^ = RN32(RN32(RN32(c / 127) * s_g) + mean), or the fp32 absmax
-        const float a = DQ ? __fadd_rn(__fmul_rn(S.inv127[cur.qa + 128], cur.sg), mu) : cur.a_raw;
-        const Lut l = build_lut(a, p.q);
-        const uint32_t wds[8] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w,
-                                 cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) lookup8(wds[i], l, v + 4 * i);
-      }
-      const int sa = ai % NS;
-      if (!mbar_wait_cluster(&S.a_empty[sa], ((ai / NS) & 1) ^ 1, abort, p.status)) break;
-      __syncwarp();
-      tc_fence_after();
-      const uint32_t taddr = tmem + tmem_lane + A_COL + sa * 32;
-      tmem_st16(taddr, v);
-      tmem_st16(taddr + 16, v + 16);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.a_full[sa]), 0));
-      cur = nxt;
-      have = more;
-      ai += 2;
-    }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
@@ -323,15 +220,15 @@ k_qlora_gemm_pair(const __grid_constant__ CUtensorMap tm_tok,     // [Mtok, Kc] 
   }
 }
 
-template <int MODE, bool DQ, int BM>
-static cudaError_t launch_pair_bm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
-                                  const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
+template <int BM>
+static cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2,
+                               const CUtensorMap& a3, const GemmArgs& a, int clusters, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_devs{0};
-  set_smem_attr_once(k_qlora_gemm_pair<MODE, DQ, BM>, (int)smem_bytes<MODE, BM>(), attr_devs);
+  set_smem_attr_once(k_qlora_gemm_pair<BM>, (int)smem_bytes<BM>(), attr_devs);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<MODE, BM>();
+  cfg.dynamicSmemBytes = smem_bytes<BM>();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -340,29 +237,19 @@ static cudaError_t launch_pair_bm(const CUtensorMap& a0, const CUtensorMap& a1, 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<MODE, DQ, BM>, a0, a1, a2, a3, a);
-}
-
-template <int BM>
-static cudaError_t launch_pair(int mode, const CUtensorMap& a0, const CUtensorMap& a1,
-                               const CUtensorMap& a2, const CUtensorMap& a3, const GemmArgs& a,
-                               int clusters, cudaStream_t s) {
-  if (mode == MODE_BF16) return launch_pair_bm<MODE_BF16, false, BM>(a0, a1, a2, a3, a, clusters, s);
-  if (a.double_quant) return launch_pair_bm<MODE_NF4, true, BM>(a0, a1, a2, a3, a, clusters, s);
-  return launch_pair_bm<MODE_NF4, false, BM>(a0, a1, a2, a3, a, clusters, s);
+  return cudaLaunchKernelEx(&cfg, k_qlora_gemm_pair<BM>, a0, a1, a2, a3, a);
 }
 
 }  // namespace pair
 
 // Token-tile width of the paired GEMM for an [Mtok x Nout] output on
 // `clusters_max` SM pairs.  A pair tile costs (fixed + width) per K step --
-// the fixed part, the A-operand supply, dominates: about 4000 width units in
-// MODE_NF4 (the converter warps) and 480 in MODE_BF16 (the weight-tile TMA),
-// as timed on B200 -- and a launch lasts as many rounds as the busiest pair
-// runs tiles.  The narrower width pays only where it removes a round.
-int pair_token_tile(int mode, int64_t Mtok, int64_t Nout, int clusters_max) {
+// the fixed part, the weight-tile TMA, is about 480 width units as timed on
+// B200 -- and a launch lasts as many rounds as the busiest pair runs tiles.
+// The narrower width pays only where it removes a round.
+static int pair_token_tile(int64_t Mtok, int64_t Nout, int clusters_max) {
   static const int kWidths[] = {256, 224};
-  const int64_t fixed = mode == MODE_NF4 ? 4000 : 480;
+  const int64_t fixed = 480;
   const int64_t n_pairs_n = (Nout + 255) / 256;
   int best = 256;
   int64_t best_cost = INT64_MAX;
@@ -376,27 +263,22 @@ int pair_token_tile(int mode, int64_t Mtok, int64_t Nout, int clusters_max) {
   return best;
 }
 
-// Paired-SM GEMM.  MODE_NF4: weights from `a` (NF4); MODE_BF16: w [Nout, Kc]
-// and wad [Nout, RP] bf16 by TMA.  Returns QLORA_OK or QLORA_ERR_CUDA.
-int launch_qlora_gemm_pair(int mode, const GemmArgs& a, const void* tok, const void* tokad,
-                           const void* wad, const void* w, int RP, cudaStream_t s, int num_sms) {
+// Paired-SM dX GEMM: w [Nout, Kc] and wad [Nout, RP] bf16 by TMA.  Returns
+// QLORA_OK or QLORA_ERR_CUDA.
+int launch_qlora_gemm_pair(const GemmArgs& a, const void* tok, const void* tokad, const void* wad,
+                           const void* w, int RP, cudaStream_t s, int num_sms) {
   using namespace pair;
-  const int bm = pair_token_tile(mode, a.Mtok, a.Nout, num_sms / 2);
+  const int bm = pair_token_tile(a.Mtok, a.Nout, num_sms / 2);
   CUtensorMap t_tok, t_tokad, t_w, t_wad;
   if (!make_tmap_2d_bf16(&t_tok, tok, a.Kc, a.Mtok, a.Kc, BK, bm / 2)) return QLORA_ERR_CUDA;
   if (!make_tmap_2d_bf16(&t_tokad, tokad, RP, a.Mtok, RP, BK, bm / 2)) return QLORA_ERR_CUDA;
-  if (mode == MODE_BF16) {
-    if (!make_tmap_2d_bf16(&t_w, w, a.Kc, a.Nout, a.Kc, BK, BN)) return QLORA_ERR_CUDA;
-    if (!make_tmap_2d_bf16(&t_wad, wad, RP, a.Nout, RP, BK, BN)) return QLORA_ERR_CUDA;
-  } else {
-    t_w = t_tok;                                   // unused
-    t_wad = t_tokad;
-  }
+  if (!make_tmap_2d_bf16(&t_w, w, a.Kc, a.Nout, a.Kc, BK, BN)) return QLORA_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&t_wad, wad, RP, a.Nout, RP, BK, BN)) return QLORA_ERR_CUDA;
   const int n_tiles = ((a.Nout + 2 * BN - 1) / (2 * BN)) * ((a.Mtok + bm - 1) / bm);
   const int clusters = std::max(1, std::min(n_tiles, num_sms / 2));
   cudaError_t e;
-  if (bm == 224) e = launch_pair<224>(mode, t_tok, t_tokad, t_w, t_wad, a, clusters, s);
-  else e = launch_pair<256>(mode, t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  if (bm == 224) e = launch_pair<224>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
+  else e = launch_pair<256>(t_tok, t_tokad, t_w, t_wad, a, clusters, s);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
