@@ -706,6 +706,26 @@ def _cores():
         return os.cpu_count() or 1
 
 
+def _host_info():
+    """The host CPU model and NumPy's BLAS, recorded beside the CPU timing."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    blas = "unknown"
+    try:
+        dep = np.show_config(mode="dicts")["Build Dependencies"]["blas"]
+        blas = f"{dep.get('name', '?')} {dep.get('version', '')}".strip()
+    except Exception:
+        pass
+    return {"cpu_model": model, "blas": blas}
+
+
 def cpu_baseline(budget_s: float):
     """Time the oracle on a sample sized to roughly `budget_s` seconds."""
     size = _calibrate(budget_s)
@@ -716,7 +736,7 @@ def cpu_baseline(budget_s: float):
     return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
             "sample": f"each projection cut to its first {size} output rows and {size} tokens: "
                       "NumPy quantise + DQ + dequantise, fp64 forward, backward, 16-token decode",
-            "seconds": el}
+            "seconds": el, **_host_info()}
 
 
 def run_reference(args, rank, world):
@@ -741,7 +761,7 @@ def run_reference(args, rank, world):
            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Gaussian)",
            "config": {"workload": "mlp_7b (sampled for the CPU oracle)", "parallelism": "none"},
            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
-                            "sample": sample},
+                            "sample": sample, **_host_info()},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
