@@ -280,21 +280,6 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[t][nt][i] = 0.f;
 
-  // scale inputs of this lane's row for a unit: DQ: int8 code and group
-  // scale; else the fp32 absmax
-  auto load_scales = [&](int rgp, int st, int& qs, float& fs) {
-    const int b = st * kBlk + j;
-    if (rgp < p.nat || b >= p.nb) return;
-    const int64_t row = min((rgp - p.nat) * kRows + srow, p.N - 1);
-    const int64_t bi = row * p.nb + b;
-    if (DQ) {
-      qs = __ldg(p.qabsmax + bi);
-      fs = __ldg(p.dq_scale + (bi >> 8));
-    } else {
-      fs = __ldg(p.absmax + bi);
-    }
-  };
-
   // sum the eight blocks' values of the current piece (in block order) and
   // write its partial
   auto flush = [&](int rgp) {
@@ -328,7 +313,6 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     consumer_sync();
   };
 
-  uint32_t k = 0;
   int cur = -1;
   bool ok = true;
   int rgp = (int)(u0 / p.spr), st = (int)(u0 - (int64_t)rgp * p.spr);
@@ -338,14 +322,31 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
   int sq[kAhead] = {0, 0, 0};
   float sf[kAhead] = {0.f, 0.f, 0.f};
   int prgp = rgp, pst = st;                       // next unit to prefetch
+  // the prefetch cursor's block index (row srow of row group prgp, block pst*8+j)
+  int64_t pbi = 0;
+  auto set_pbi = [&]() {
+    pbi = (int64_t)min((prgp - p.nat) * kRows + srow, p.N - 1) * p.nb + pst * kBlk + j;
+  };
+  set_pbi();
+  auto load_next = [&](int& qs_, float& fs_) {
+    if (prgp >= p.nat && pst * kBlk + j < p.nb) {
+      if (DQ) {
+        qs_ = __ldg(p.qabsmax + pbi);
+        fs_ = __ldg(p.dq_scale + (pbi >> 8));
+      } else {
+        fs_ = __ldg(p.absmax + pbi);
+      }
+    }
+    if (++pst == p.spr) { pst = 0; ++prgp; set_pbi(); }
+    else pbi += kBlk;
+  };
+  const int L = (int)(u1 - u0);
 #pragma unroll
-  for (int d = 0; d < kAhead; ++d) {
-    if (u0 + d < u1) load_scales(prgp, pst, sq[d], sf[d]);
-    if (++pst == p.spr) { pst = 0; ++prgp; }
-  }
+  for (int d = 0; d < kAhead; ++d)
+    if (d < L) load_next(sq[d], sf[d]);
   int s = 0;
   uint32_t ph = 0;                               // phase of stage s's current use
-  for (int64_t u = u0; u < u1; ++u, ++k, s = (s + 1 == kStages) ? 0 : s + 1, ph ^= (s == 0)) {
+  for (int i = 0; i < L; ++i, s = (s + 1 == kStages) ? 0 : s + 1, ph ^= (s == 0)) {
     const int b = st * kBlk + j;
     int nrgp = rgp, nst = st + 1;                 // the next unit
     if (nst == p.spr) { nst = 0; ++nrgp; }
@@ -357,8 +358,7 @@ k_qlora_gemv(const __grid_constant__ CUtensorMap tm_codes,   // packed [N, K/2] 
     const float fs = sf[0];
 #pragma unroll
     for (int d = 0; d + 1 < kAhead; ++d) { sq[d] = sq[d + 1]; sf[d] = sf[d + 1]; }
-    if (u + kAhead < u1) load_scales(prgp, pst, sq[kAhead - 1], sf[kAhead - 1]);
-    if (++pst == p.spr) { pst = 0; ++prgp; }
+    if (i + kAhead < L) load_next(sq[kAhead - 1], sf[kAhead - 1]);
     if (!(ok = mbar_wait(&S.full[s], ph, abort, p.status))) break;
     const uint8_t* sb = stage_ptr(s);
     const bool nf4 = rgp >= p.nat;
