@@ -18,10 +18,10 @@
 namespace qnf4 {
 
 // ===========================================================================
-// Quantise: one thread owns one 64-weight block at a time (eight 16-byte
-// bf16 loads or sixteen fp32 ones, a 32-byte code store and its absmax), so
-// the block max, the reciprocal and the stores cost one thread's work per 64
-// weights, and a warp's 32 blocks are contiguous.  A persistent grid (two
+// Quantise: a 64-weight block belongs to two threads (bf16 input: 32
+// weights, four 16-byte loads and a 16-byte code store each) or four (fp32
+// input: 16 weights, an 8-byte store); the block max takes one or two
+// shuffles, and a warp's blocks are contiguous.  A persistent grid (three
 // CTAs per SM) walks the blocks; each thread loads its next block's words
 // before it computes the current block's codes.  absmax is an integer max over |w| bit
 // patterns (exact; NaN/Inf show up as >= 0x7f800000).
@@ -76,10 +76,31 @@ __device__ __forceinline__ uint32_t code_of(float x, uint32_t lane_base, uint32_
   return up ? (b.codes >> 8) : (b.codes & 0xFFu);
 }
 
-// Weight i (0..63) of a block as an fp32 bit pattern, from the block's words.
-template <typename T> struct BlockWords;
-template <> struct BlockWords<__nv_bfloat16> {
-  static constexpr int kWords = 32;               // bf16 pairs, element 2j in the low half
+// Threads that share one 64-weight block, and CTAs per SM: every thread
+// holds 64 bytes of input (four 16-byte loads), so a bf16 block is split
+// between two threads and an fp32 block between four; three CTAs per SM.
+// Smaller parts give an SM more warps over the same bytes in flight.
+template <typename T> struct QuantShape;
+template <> struct QuantShape<__nv_bfloat16> { static constexpr int kTPB = 2, kCTAs = 3; };
+template <> struct QuantShape<float> { static constexpr int kTPB = 4, kCTAs = 3; };
+
+// Store N code words (N = 2, 4 or 8) at a 4N-byte aligned address.
+template <int N>
+__device__ __forceinline__ void store_code_words(uint8_t* dst, const uint32_t (&out)[N]) {
+  if constexpr (N == 2) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q)
+      reinterpret_cast<uint4*>(dst)[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  }
+}
+
+// Weight i of a thread's part of a block as an fp32 bit pattern, from the
+// part's words, and the part's max |w| bit pattern.
+template <typename T> struct PartWords;
+template <> struct PartWords<__nv_bfloat16> {
+  static constexpr int kWords = 32 / QuantShape<__nv_bfloat16>::kTPB;   // bf16 pairs, element 2j in the low half
   __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) {
     return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
   }
@@ -91,8 +112,8 @@ template <> struct BlockWords<__nv_bfloat16> {
     return max(mm << 16, mm & 0xFFFF0000u);
   }
 };
-template <> struct BlockWords<float> {
-  static constexpr int kWords = 64;
+template <> struct PartWords<float> {
+  static constexpr int kWords = 64 / QuantShape<float>::kTPB;
   __device__ __forceinline__ static uint32_t elem(const uint32_t (&w)[kWords], int i) { return w[i]; }
   __device__ __forceinline__ static uint32_t absmax_bits(const uint32_t (&w)[kWords]) {
     uint32_t m = 0;
@@ -102,37 +123,40 @@ template <> struct BlockWords<float> {
   }
 };
 
-// Exact codes of block `blk` (x = RN32(w / a), or 0 for a zero block),
-// written straight to `packed`: the rare path, kept out of line so the hot
-// loop keeps its registers.
+// Exact codes of part `part` of block `blk` (weights [part * kW, +kW); x =
+// RN32(w / a), or 0 for a zero block), written straight to `packed`: the rare
+// path, kept out of line so the hot loop keeps its registers.
 template <typename T, bool MONO>
-__device__ __noinline__ void exact_block_codes(const void* W, int64_t blk, float a, bool zero_block,
-                                               uint32_t lane_base, uint8_t* packed) {
-  uint32_t out[8];
+__device__ __noinline__ void exact_part_codes(const void* W, int64_t blk, int part, float a,
+                                              bool zero_block, uint32_t lane_base, uint8_t* packed) {
+  constexpr int kW = 64 / QuantShape<T>::kTPB;
+  uint32_t out[kW / 8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) out[k] = 0u;
+  for (int k = 0; k < kW / 8; ++k) out[k] = 0u;
   uint32_t unused = 0;
-  for (int i = 0; i < 64; ++i) {
+  for (int i = 0; i < kW; ++i) {
+    const int64_t idx = blk * 64 + part * kW + i;
     float w;
-    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[blk * 64 + i]);
-    else w = reinterpret_cast<const float*>(W)[blk * 64 + i];
+    if (sizeof(T) == 2) w = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(W)[idx]);
+    else w = reinterpret_cast<const float*>(W)[idx];
     const float x = zero_block ? 0.0f : __fdiv_rn(w, a);
     const uint32_t code = code_of<MONO>(x, lane_base, unused);
     const int sh = 8 * ((i >> 1) & 3) + ((i & 1) ? 0 : 4);
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < kW / 8; ++k)
       if (k == (i >> 3)) out[k] |= code << sh;
   }
-  uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
-  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  store_code_words(packed + blk * 32 + part * (kW / 2), out);
 }
 
 template <typename T, bool MONO, bool HIST>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, QuantShape<T>::kCTAs)
 k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packed,
            float* __restrict__ absmax, unsigned long long* __restrict__ hist, CodeTables tb,
            int* status) {
+  constexpr int kTPB = QuantShape<T>::kTPB;
+  constexpr int kWords = PartWords<T>::kWords;   // 32-bit words of a thread's part
+  constexpr int kOut = 8 / kTPB;                 // code words of a part
   __shared__ __align__(8) Bucket s_bk[64 * 32];  // bucket b, lane l at b * 32 + l
   __shared__ unsigned long long s_hist[HIST ? 256 : 1];
   for (int i = threadIdx.x; i < 64 * 32; i += blockDim.x) {
@@ -144,18 +168,19 @@ k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packe
     for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0ull;
   __syncthreads();
   const int lane = threadIdx.x & 31;
+  const int pb = lane / kTPB, part = lane % kTPB;   // block of the warp's 32 / kTPB, part of it
   const uint32_t lane_base = smem_u32(s_bk) + (uint32_t)lane * 8u;
-  constexpr int kWords = BlockWords<T>::kWords;
   bool bad = false;
   // warp-uniform loop (the histogram's match/reduce need whole warps); the
   // next block's words are loaded before this block's codes are computed
-  const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  const int64_t gstride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t first = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) / kTPB;
+  const int64_t gstride = (int64_t)gridDim.x * blockDim.x / kTPB;
   uint32_t wn[kWords];
   auto load_words = [&](int64_t base_) {
-    const int64_t b = base_ + lane;
+    const int64_t b = base_ + pb;
     const bool v_ = b < nblk;
-    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords / 4) * (v_ ? b : 0);
+    const uint4* src = reinterpret_cast<const uint4*>(W) + (int64_t)(kWords * kTPB / 4) * (v_ ? b : 0) +
+                       (kWords / 4) * part;
 #pragma unroll
     for (int k = 0; k < kWords / 4; ++k) {
       const uint4 v = v_ ? __ldcs(src + k) : make_uint4(0u, 0u, 0u, 0u);
@@ -164,43 +189,43 @@ k_quantize(const void* __restrict__ W, int64_t nblk, uint8_t* __restrict__ packe
   };
   if (first < nblk) load_words(first);
   for (int64_t base = first; base < nblk; base += gstride) {
-    const int64_t blk = base + lane;
+    const int64_t blk = base + pb;
     const bool valid = blk < nblk;
     uint32_t w[kWords];
 #pragma unroll
     for (int k = 0; k < kWords; ++k) w[k] = wn[k];
     if (base + gstride < nblk) load_words(base + gstride);
-    uint32_t m = BlockWords<T>::absmax_bits(w);
+    uint32_t m = PartWords<T>::absmax_bits(w);
+#pragma unroll
+    for (int o = 1; o < kTPB; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (m >= 0x7F800000u) { bad = true; m = 0; }
     const float a = __uint_as_float(m);
     if (valid) {
       const bool exact_block = m < 0x01000000u;   // a == 0 or a < 2^-125
       const float inv = exact_block ? 0.0f : rcp_approx(a);
-      uint32_t out[8];
-      uint32_t nearm = 0xFFFFFFFFu;               // min over the block of (ulp distance to T) + 8
+      uint32_t out[kOut];
+      uint32_t nearm = 0xFFFFFFFFu;               // min over the part of (ulp distance to T) + 8
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kOut; ++k) {
         uint32_t o = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int i = 8 * k + e;
-          const float x = __fmul_rn(__uint_as_float(BlockWords<T>::elem(w, i)), inv);
+          const float x = __fmul_rn(__uint_as_float(PartWords<T>::elem(w, i)), inv);
           // element 2j -> high nibble of byte j (fields disjoint: add = or)
           o += code_of<MONO>(x, lane_base, nearm) << (8 * (e >> 1) + ((e & 1) ? 0 : 4));
         }
         out[k] = o;
       }
       if (exact_block || nearm <= 16u) {
-        exact_block_codes<T, MONO>(W, blk, a, m == 0, lane_base, packed);
+        exact_part_codes<T, MONO>(W, blk, part, a, m == 0, lane_base, packed);
       } else {
-        uint4* dst = reinterpret_cast<uint4*>(packed) + 2 * blk;
-        dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        store_code_words(packed + blk * 32 + part * (kOut * 4), out);
       }
-      absmax[blk] = a;
+      if (part == 0) absmax[blk] = a;
     }
     if (HIST) {
-      const bool add = valid && m != 0u;
+      const bool add = valid && m != 0u && part == 0;
       const uint32_t e = add ? (m >> 23) : 0xFFFFFFFFu;
       const uint32_t mant = add ? ((m & 0x7FFFFFu) | (e ? 0x800000u : 0u)) : 0u;
       const uint32_t grp = __match_any_sync(0xffffffffu, e);
@@ -221,12 +246,13 @@ static void launch_quantize_t(const void* W, int64_t nblk, uint8_t* packed, floa
                               unsigned long long* hist, const CodeTables& tb, int* status,
                               cudaStream_t s) {
   constexpr int kThreads = 256;
-  // one block per thread: other CTAs' loads cover each block's compute
+  constexpr int kTPB = QuantShape<T>::kTPB;
+  // persistent grid: kCTAs per SM; other CTAs' loads cover each block's compute
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nblk + kThreads - 1) / kThreads,
-                                                                 (int64_t)sms * 2));
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nblk * kTPB + kThreads - 1) / kThreads,
+                                                                 (int64_t)sms * QuantShape<T>::kCTAs));
   if (hist)
     k_quantize<T, MONO, true><<<blocks, kThreads, 0, s>>>(W, nblk, packed, absmax, hist, tb, status);
   else
