@@ -166,6 +166,31 @@ def test_edge_values(q):
         _check_full(q, Wt, False, FP4)
 
 
+@pytest.mark.parametrize("qt", [NF4, FP4])
+def test_threshold_values_every_part(q, qt):
+    # fp32 blocks whose absmax is exactly 1, with the weights T - 1 ulp, T and
+    # T + 1 ulp (T a decision threshold of the table) placed in one of the
+    # threads' parts of each block, part by part: the quotient lands within a
+    # few ulp of T, so that part is coded by the exact (IEEE division) path
+    # and the block's other parts by the fast path; ties go up.
+    rng = np.random.default_rng(33)
+    thr = oracle.thresholds(_table(qt))
+    W = (rng.standard_normal((24, 512)) * 0.1).clip(-0.5, 0.5).astype(np.float32)
+    nblk = W.size // 64
+    Wb = W.reshape(nblk, 64)
+    for b in range(nblk):
+        Wb[b, 63 - (b % 7)] = 1.0 if b % 2 else -1.0          # the block's absmax
+        T = thr[b % thr.size]
+        part = b % 4                                            # a 16-weight part
+        lo = part * 16 + 3
+        Wb[b, lo] = np.nextafter(T, np.float32(-np.inf))
+        Wb[b, lo + 1] = T
+        Wb[b, lo + 2] = np.nextafter(T, np.float32(np.inf))
+    Wt = torch.from_numpy(Wb.reshape(W.shape).copy())
+    _check_full(q, Wt, True, qt)
+    _check_full(q, Wt, False, qt)
+
+
 def test_nonfinite_sets_status(q):
     W = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
     W[2, 5] = float("nan")
