@@ -16,10 +16,11 @@
 //    partial per output, and the pieces of a row group belong to consecutive
 //    CTAs.
 //  * One producer warp streams the CTA's units through a ring of TMA stages
-//    (five for one token tile, three for two), two or three copies per stage: the codes as two 64-row x 128-byte
-//    boxes (128B-swizzled: wide rows, conflict-free reads) or the 8 blocks of
-//    16 rows of A as one 3-D box, and the tokens' 8 blocks of X as one 3-D
-//    box (8 or 16 rows x 64 per block, 128B-swizzled).
+//    (five for one token tile, three for two), two or three copies per
+//    stage: the codes as two 64-row x 128-byte boxes (128B-swizzled: wide
+//    rows, conflict-free reads) or the 8 blocks of 16 rows of A as one 3-D
+//    box, and the tokens' 8 blocks of X as one 3-D box (8 or 16 rows x 64
+//    per block, 128B-swizzled).
 //  * Sixteen consumer warps: warp (j, h) takes NF4 block j of the stage for
 //    rows [32h, 32h+32) as two 16-row tiles of mma.m16n8k16 (tokens are the
 //    8-column operand, one or two tiles).
